@@ -1,0 +1,279 @@
+/*
+ * oracle.c -- plain fp64 CPU oracle for bitmask-driven block-sparse attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only tests/, the smoke check and the bench's CPU-baseline
+ * leg use it.  It shares no code, header or constant with the CUDA library.
+ *
+ * What it computes, and where the pages define it:
+ *
+ *  - CRM (Compressed Row Mask): one bitmask row per query block, stored as
+ *    uint32 words, one bit per key block ("ScalingAttention", Sec. 4.3.2).
+ *    The bit order follows the forward iterator of Appendix E (Algorithm 2):
+ *    the iterator's base starts at -32 and grows by 32 per word loaded, and
+ *    the block index is base + count-trailing-zeros, so bit j of word w is
+ *    key block 32*w + j.
+ *  - The CRM forward iterator itself (Init / Advance / Next / Index,
+ *    Appendix E, Algorithm 2), used here to list the kept key blocks of a row.
+ *  - Masked softmax attention: the block-sparse FlashAttention forward of
+ *    Sec. 4.3.2 computes, for every query, softmax over the keys of the kept
+ *    blocks only; a masked block contributes exp(-inf) = 0.  We write out the
+ *    plain definition: s = scale * q.k, -inf where the block is masked,
+ *    m = max s, l = sum exp(s - m), o = sum exp(s - m) v / l, lse = m + ln l.
+ *  - The 3-D tile permutation (token reordering, Sec. 5.4-5.5): tiles are
+ *    enumerated (tile_t, tile_y, tile_x) row-major; inside a tile the tokens
+ *    go (t, y, x) row-major over the tile's clipped extent; tokens are
+ *    concatenated with no holes and the tail is zero-padded.
+ *
+ * Everything is fp64 except the inputs, which arrive as raw bf16 bits and are
+ * widened exactly to double.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ */
+/* bf16 -> double, exact                                               */
+/* ------------------------------------------------------------------ */
+static double bf16_bits_to_double(uint16_t b) {
+  uint32_t u = ((uint32_t)b) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------ */
+/* CRM words per row: one uint32 holds the state of 32 key blocks      */
+/* (ScalingAttention Sec. 4.3.2).                                      */
+/* ------------------------------------------------------------------ */
+int oracle_crm_words(int nb_k) { return (nb_k + 31) / 32; }
+
+/* Dense 0/1 block mask rows -> CRM bit rows.  A nonzero byte is a kept
+ * block.  rows = B*H*nb_q; dense is [rows, nb_k]; bits is [rows, words]. */
+void oracle_pack_bits(const uint8_t* dense, int64_t rows, int nb_k, uint32_t* bits) {
+  int words = oracle_crm_words(nb_k);
+  for (int64_t r = 0; r < rows; ++r) {
+    uint32_t* row_bits = bits + r * words;
+    for (int w = 0; w < words; ++w) row_bits[w] = 0u;
+    for (int j = 0; j < nb_k; ++j) {
+      if (dense[r * (int64_t)nb_k + j] != 0) {
+        row_bits[j / 32] |= (1u << (j % 32));
+      }
+    }
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* CRM forward iterator, ScalingAttention Appendix E (Algorithm 2).    */
+/* State {ptr, end, val, base}.                                        */
+/* ------------------------------------------------------------------ */
+typedef struct {
+  const uint32_t* ptr;
+  const uint32_t* end;
+  uint32_t val;
+  int64_t base;
+} crm_iterator;
+
+/* Skip empty segments: load words until one is nonzero or the row ends. */
+static void crm_advance(crm_iterator* s) {
+  while (s->val == 0u && s->ptr != s->end) {
+    s->val = *s->ptr;
+    s->ptr += 1;
+    s->base += 32;
+  }
+}
+
+static void crm_init(crm_iterator* s, const uint32_t* row_ptr, int n_words) {
+  s->ptr = row_ptr;
+  s->end = row_ptr + n_words;
+  s->val = 0u;
+  s->base = -32;
+  crm_advance(s); /* prefetch the first nonzero segment */
+}
+
+/* Consume the current active block: clear the lowest set bit. */
+static void crm_next(crm_iterator* s) {
+  s->val = s->val & (s->val - 1u);
+  if (s->val == 0u) crm_advance(s);
+}
+
+static int count_trailing_zeros(uint32_t v) {
+  int n = 0;
+  while ((v & 1u) == 0u) {
+    v >>= 1;
+    n += 1;
+  }
+  return n;
+}
+
+/* Global key-block index of the current active block, -1 for the end-of-row
+ * sentinel. */
+static int64_t crm_index(const crm_iterator* s) {
+  if (s->val == 0u) return -1;
+  return s->base + count_trailing_zeros(s->val);
+}
+
+/* Walk every CRM row with the iterator: counts[r] = number of kept blocks,
+ * row_offsets = exclusive prefix of counts (rows+1 entries), col_idx = the
+ * kept block indices of each row in the order the iterator yields them.
+ * col_idx may be NULL to only count.  Returns the total. */
+int64_t oracle_crm_lists(const uint32_t* bits, int64_t rows, int n_words, int32_t* counts,
+                         int64_t* row_offsets, int32_t* col_idx) {
+  int64_t total = 0;
+  for (int64_t r = 0; r < rows; ++r) {
+    crm_iterator it;
+    crm_init(&it, bits + r * n_words, n_words);
+    int64_t c = 0;
+    row_offsets[r] = total;
+    for (int64_t j = crm_index(&it); j != -1; crm_next(&it), j = crm_index(&it)) {
+      if (col_idx) col_idx[total + c] = (int32_t)j;
+      c += 1;
+    }
+    counts[r] = (int32_t)c;
+    total += c;
+  }
+  row_offsets[rows] = total;
+  return total;
+}
+
+/* Schedule: row ids ordered by kept-block count, largest first; rows with
+ * equal counts keep ascending row order.  Written as the plainest counting
+ * order: for each count value from the largest down, list its rows. */
+void oracle_schedule(const int32_t* counts, int64_t rows, int32_t* schedule) {
+  int32_t max_count = 0;
+  for (int64_t r = 0; r < rows; ++r)
+    if (counts[r] > max_count) max_count = counts[r];
+  int64_t pos = 0;
+  for (int32_t c = max_count; c >= 0; --c)
+    for (int64_t r = 0; r < rows; ++r)
+      if (counts[r] == c) schedule[pos++] = (int32_t)r;
+}
+
+/* ------------------------------------------------------------------ */
+/* 3-D tile permutation.  perm[p] = frame-major token index (t*H + y)*W */
+/* + x of the token stored at tile-major position p, p < T*H*W.        */
+/* ------------------------------------------------------------------ */
+static int min_int(int a, int b) { return a < b ? a : b; }
+
+void oracle_tile_order(int T, int Hs, int Ws, int tt, int th, int tw, int64_t* perm) {
+  int64_t p = 0;
+  for (int t0 = 0; t0 < T; t0 += tt)
+    for (int y0 = 0; y0 < Hs; y0 += th)
+      for (int x0 = 0; x0 < Ws; x0 += tw) {
+        int t1 = min_int(t0 + tt, T), y1 = min_int(y0 + th, Hs), x1 = min_int(x0 + tw, Ws);
+        for (int t = t0; t < t1; ++t)
+          for (int y = y0; y < y1; ++y)
+            for (int x = x0; x < x1; ++x) perm[p++] = ((int64_t)t * Hs + y) * Ws + x;
+      }
+}
+
+/* Gather rows of d bf16 values: out[bh, p, :] = in[bh, perm[p], :] for
+ * p < n, zero for n <= p < n_pad.  in is [BH, n, d], out is [BH, n_pad, d]. */
+void oracle_permute(const uint16_t* in, uint16_t* out, int64_t BH, int64_t n, int64_t n_pad,
+                    int d, const int64_t* perm) {
+  for (int64_t bh = 0; bh < BH; ++bh)
+    for (int64_t p = 0; p < n_pad; ++p) {
+      uint16_t* dst = out + (bh * n_pad + p) * d;
+      if (p < n) {
+        const uint16_t* src = in + (bh * n + perm[p]) * d;
+        memcpy(dst, src, (size_t)d * sizeof(uint16_t));
+      } else {
+        memset(dst, 0, (size_t)d * sizeof(uint16_t));
+      }
+    }
+}
+
+/* Inverse: out[bh, perm[p], :] = in[bh, p, :] for p < n; pad rows dropped. */
+void oracle_unpermute(const uint16_t* in, uint16_t* out, int64_t BH, int64_t n, int64_t n_pad,
+                      int d, const int64_t* perm) {
+  for (int64_t bh = 0; bh < BH; ++bh)
+    for (int64_t p = 0; p < n; ++p)
+      memcpy(out + (bh * n + perm[p]) * d, in + (bh * n_pad + p) * d,
+             (size_t)d * sizeof(uint16_t));
+}
+
+/* ------------------------------------------------------------------ */
+/* Masked softmax attention in fp64.                                    */
+/*                                                                      */
+/* q, k, v: raw bf16 bits, [B*H, n_pad, d] in permuted token order.     */
+/* mask: [B*H, nb, nb] bytes, nb = n_pad / block, nonzero = kept.       */
+/* rows: the flat query ids (bh * n_pad + i) to compute, or NULL for    */
+/* all B*H*n_pad of them; n_rows their number.                          */
+/* dense_literal = 1: score every valid key and put -inf on masked      */
+/* blocks (the definition, literally).  0: visit only kept blocks,      */
+/* which is the same result because exp(-inf) = 0.                      */
+/* Outputs: out [n_rows, d], lse [n_rows].  Rows with no valid kept key */
+/* and pad rows (i >= n_valid) give out = 0, lse = -inf.                */
+/* ------------------------------------------------------------------ */
+void oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                      const uint8_t* mask, int64_t BH, int64_t n_valid, int64_t n_pad, int d,
+                      int block, double scale, const int64_t* rows, int64_t n_rows,
+                      int dense_literal, double* out, double* lse) {
+  const int64_t nb = n_pad / block;
+  if (rows == NULL) n_rows = BH * n_pad;
+
+#pragma omp parallel
+  {
+    double* s = (double*)malloc((size_t)n_valid * sizeof(double));
+    double* qi = (double*)malloc((size_t)d * sizeof(double));
+#pragma omp for schedule(dynamic, 16)
+    for (int64_t r = 0; r < n_rows; ++r) {
+      int64_t flat = rows ? rows[r] : r;
+      int64_t bh = flat / n_pad, i = flat % n_pad;
+      double* o = out + r * d;
+      for (int c = 0; c < d; ++c) o[c] = 0.0;
+      lse[r] = -INFINITY;
+      if (i >= n_valid) continue; /* pad query row */
+
+      const uint16_t* qrow = q + (bh * n_pad + i) * d;
+      for (int c = 0; c < d; ++c) qi[c] = bf16_bits_to_double(qrow[c]);
+      const uint8_t* mrow = mask + (bh * nb + i / block) * nb;
+
+      /* scores s_j for j < n_valid; -inf where the key block is masked */
+      double m = -INFINITY;
+      for (int64_t j = 0; j < n_valid; ++j) {
+        int kept = mrow[j / block] != 0;
+        if (!kept) {
+          s[j] = -INFINITY;
+          if (!dense_literal) { /* skip the rest of this masked block */
+            int64_t jend = (j / block + 1) * block;
+            for (int64_t jj = j + 1; jj < jend && jj < n_valid; ++jj) s[jj] = -INFINITY;
+            j = jend - 1;
+          }
+          continue;
+        }
+        const uint16_t* krow = k + (bh * n_pad + j) * d;
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += qi[c] * bf16_bits_to_double(krow[c]);
+        s[j] = scale * dot;
+        if (s[j] > m) m = s[j];
+      }
+      if (m == -INFINITY) continue; /* no kept key: zero output, lse = -inf */
+
+      double l = 0.0;
+      for (int64_t j = 0; j < n_valid; ++j) {
+        if (s[j] == -INFINITY) continue; /* exp(-inf - m) = 0 */
+        double p = exp(s[j] - m);
+        l += p;
+        const uint16_t* vrow = v + (bh * n_pad + j) * d;
+        for (int c = 0; c < d; ++c) o[c] += p * bf16_bits_to_double(vrow[c]);
+      }
+      for (int c = 0; c < d; ++c) o[c] /= l;
+      lse[r] = m + log(l);
+    }
+    free(s);
+    free(qi);
+  }
+}
