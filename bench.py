@@ -1,0 +1,384 @@
+"""Benchmark of the block-sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = the whole hot path over one batch of synthetic, seeded inputs that
+are already resident in HBM: bsa_pack_mask (CRM rows, lists, schedule),
+bsa_tile_permute of q, k, v, bsa_forward, bsa_tile_unpermute of the output.
+
+metric: effective TFLOPS = 4 * d * block^2 * (kept tiles) / time, with the
+step time as denominator for `value` and the forward kernel's own time for
+`roofline.achieved`.  Inputs (3 x 774 MB for the default workload) are larger
+than L2, so no flush is needed between steps.
+
+With N > 1 (torchrun), every rank runs its own independent problem of the same
+shape (different seed): the path shards by (batch, head) with no exchange, so
+there is no collective on the data path (weak scaling); the step time is the
+max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of query blocks of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_forward_b200 import inputs as I  # noqa: E402
+
+METRIC = "effective TFLOPS of bsa_forward on kept tiles and % of B200 bf16 peak"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "wan14b_720p"  # the ~75 %-sparse 720p shape the target is quoted on
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a window."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=5)
+
+    def summary(self, t0: float, t1: float):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if not (t0 <= ts <= t1):
+                continue
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_selector(dev: torch.device) -> str:
+    """nvidia-smi -i argument for this device (PCI bus id, else the CUDA index)."""
+    try:
+        pr = torch.cuda.get_device_properties(dev)
+        return f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+    except Exception:  # noqa: BLE001 - older torch without PCI fields
+        return str(dev.index or 0)
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def _bits(x: torch.Tensor) -> np.ndarray:
+    return x.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def oracle_sample(w, q, k, v, mask, budget_s: float, seed: int):
+    """Times the oracle on whole query blocks (all rows) of the workload until
+    about budget_s of CPU work; returns (tflops_equivalent, seconds, blocks, cores)."""
+    import oracle
+    BH = w.B * w.H
+    perm = oracle.tile_order(w.T, w.Hs, w.Ws, w.tt, w.th, w.tw)
+    m = mask.reshape(BH, w.nb, w.nb)
+    rng = np.random.default_rng(seed)
+    heads = rng.choice(BH, size=min(BH, 4), replace=False)
+    flat = [x.reshape(BH, w.n, w.d) for x in (q, k, v)]
+    per_head = {}
+    for bh in heads:
+        bh = int(bh)
+        per_head[bh] = tuple(oracle.permute(_bits(x[bh:bh + 1]), perm, w.n_pad) for x in flat)
+    flops = 0.0
+    spent = 0.0
+    blocks = 0
+    order = [(int(bh), int(qb)) for qb in rng.permutation(w.nb) for bh in heads]
+    for bh, qb in order:
+        qp, kp, vp = per_head[bh]
+        rows = (qb * w.block + np.arange(w.block)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attention(qp, kp, vp, m[bh:bh + 1], w.n, w.block, rows=rows)
+        spent += time.perf_counter() - t0
+        flops += 4.0 * w.d * w.block * w.block * float(m[bh, qb].sum())
+        blocks += 1
+        if spent >= budget_s:
+            break
+    return flops / spent / 1e12, spent, blocks, oracle.num_threads()
+
+
+def run_reference(args, w):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    q, k, v = I.gen_qkv(w)
+    mask = I.gen_mask(w, q, k)
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        tf, spent, blocks, cores = oracle_sample(w, q, k, v, mask, per_step, seed=w.seed + i)
+        if i >= args.warmup:
+            vals.append((tf, spent, blocks))
+    value = statistics.median([x[0] for x in vals])
+    sample = (f"fp64 C oracle (OpenMP) on whole query blocks of 4 seeded heads, about "
+              f"{per_step:.0f} s per step ({vals[0][2]} blocks of {w.block} rows in step 1)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * statistics.median([x[1] for x in vals]),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, mask),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, mask):
+    kept = I.kept_tiles(mask)
+    total = w.B * w.H * w.nb * w.nb
+    return {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "grid": [w.T, w.Hs, w.Ws],
+            "tile": [w.tt, w.th, w.tw], "block": w.block, "n_tokens": w.n, "n_pad": w.n_pad,
+            "kept_tiles": kept, "density": kept / total, "mask": w.mask_kind,
+            "l2": "inputs larger than L2 (no flush)", "parallelism": "independent problems per rank"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    w = I.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import block_sparse_attention_forward_b200 as bsa
+    from block_sparse_attention_forward_b200 import _ffi
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    seed = w.seed + 7919 * rank
+    q, k, v = I.gen_qkv(w, seed=seed)
+    mask = I.gen_mask(w, q, k, seed=seed)
+    flops = I.effective_flops(w, mask)
+    grid, tile = (w.T, w.Hs, w.Ws), (w.tt, w.th, w.tw)
+
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    maskd = torch.from_numpy(mask).to(dev)
+    qp = torch.empty((w.B, w.H, w.n_pad, w.d), dtype=torch.bfloat16, device=dev)
+    kp, vp, out_p = torch.empty_like(qp), torch.empty_like(qp), torch.empty_like(qp)
+    out = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.H, w.n_pad), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    fwd_ev = []
+
+    def step(record_fwd: bool):
+        pm = bsa.pack_mask(maskd)
+        bsa.tile_permute(qd, grid, tile, w.n_pad, out=qp)
+        bsa.tile_permute(kd, grid, tile, w.n_pad, out=kp)
+        bsa.tile_permute(vd, grid, tile, w.n_pad, out=vp)
+        if record_fwd:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        bsa.forward(qp, kp, vp, pm, w.n, w.block, out=out_p, lse=lse)
+        if record_fwd:
+            e1.record(stream)
+            fwd_ev.append((e0, e1))
+        bsa.tile_unpermute(out_p, grid, tile, out=out)
+        return pm
+
+    launches_per_step = 3 + 3 + 1 + 1  # pack (3), permute q/k/v, forward, unpermute
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize(dev)
+    if bsa.device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    sampler = ClockSampler(gpu_selector(dev))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step(True)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    sampler.stop()
+    ms_total = ev0.elapsed_time(ev1)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev)
+    if bsa.device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+
+    t = torch.tensor([ms_total, fwd_ms, flops], dtype=torch.float64, device=dev)
+    total_flops = flops
+    if world > 1:
+        tmax = t[:2].clone()
+        torch.distributed.all_reduce(tmax, op=torch.distributed.ReduceOp.MAX)
+        tf = t[2:].clone()
+        torch.distributed.all_reduce(tf, op=torch.distributed.ReduceOp.SUM)
+        ms_total, fwd_ms = float(tmax[0]), float(tmax[1])
+        total_flops = float(tf[0])
+    ms_step = ms_total / args.steps
+    value = total_flops / (ms_step * 1e-3) / 1e12
+
+    # ---------------------------------------------------------------- e2e
+    e2e = None
+    if not args.no_e2e:
+        lib = _ffi.load()
+        h_q, h_k, h_v = q.pin_memory(), k.pin_memory(), v.pin_memory()
+        h_mask = torch.from_numpy(mask).pin_memory()
+        h_out = torch.empty_like(q).pin_memory()
+        h_lse = torch.empty((w.B, w.H, w.n_pad), dtype=torch.float32).pin_memory()
+        e_steps = max(2, min(args.steps, 5))
+        sp = ctypes.c_void_p(stream.cuda_stream)
+
+        def e2e_step():
+            qd.copy_(h_q, non_blocking=True)
+            kd.copy_(h_k, non_blocking=True)
+            vd.copy_(h_v, non_blocking=True)
+            maskd.copy_(h_mask, non_blocking=True)
+            step(False)
+            h_out.copy_(out, non_blocking=True)
+            h_lse.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = a0.elapsed_time(a1) / e_steps
+        te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+        e_ms = float(te[0])
+        h2d = sum(x.numel() * x.element_size() for x in (h_q, h_k, h_v, h_mask))
+        d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
+        e2e = {"value": total_flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del sp
+
+    # ---------------------------------------------------------------- roofline
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
+                "frac": fwd_tflops / peak, "traffic": None, "kernel": "bsa_forward_kernel<128,128>",
+                "peak_source": f"{peak_src} bf16_tflops_sustained (dense bf16 cuBLAS, seconds-long loop)",
+                "fwd_ms": fwd_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, spent, blocks, cores = oracle_sample(w, q, k, v, mask, 15.0, seed=w.seed)
+        cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{blocks} whole query blocks ({w.block} rows each) of 4 seeded heads, "
+                         f"{spent:.1f} s of fp64 OpenMP oracle"}
+
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 q/k/v, PSA-style stripe masks)",
+            "config": workload_config(w, mask), "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+            "clocks": sampler.summary(t_wall0, t_wall1),
+            "peak_frac_step": value / peak,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,156 @@
+"""bitmask-driven block-sparse attention forward for B200 (sm_100a).
+
+Torch-facing wrappers over the C ABI of libbsa (include/bsa.h).  PyTorch only
+provides device memory and the current stream; each call checks dtypes,
+devices and contiguity, then passes raw pointers to the library.
+
+    mask = pack_mask(dense_u8)                     # CRM rows, lists, schedule
+    qp = tile_permute(q, grid, tile, n_pad)        # frame-major -> 3-D tiles
+    out_p, lse = forward(qp, kp, vp, mask, n_valid, block)
+    out = tile_unpermute(out_p, grid, tile)        # back to frame-major
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _ffi
+from ._ffi import BsaError, BsaMask
+
+__all__ = ["BsaError", "PackedMask", "pack_mask", "tile_permute", "tile_unpermute", "forward",
+           "device_error", "version"]
+
+
+def _stream(device: torch.device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _require_cuda(t: torch.Tensor, name: str, dtype: torch.dtype | None = None) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def version() -> int:
+    return _ffi.load().bsa_version()
+
+
+@dataclass
+class PackedMask:
+    """Device tensors produced by bsa_pack_mask (see include/bsa.h)."""
+    bits: torch.Tensor         # uint32 as int32 [B, H, nb_q, words]
+    counts: torch.Tensor       # int32 [B*H*nb_q]
+    row_offsets: torch.Tensor  # int32 [B*H*nb_q + 1]
+    col_idx: torch.Tensor | None  # int32 [B*H*nb_q*nb_k] (valid prefix row_offsets[-1])
+    schedule: torch.Tensor     # int32 [B*H*nb_q]
+    B: int
+    H: int
+    nb_q: int
+    nb_k: int
+
+    @property
+    def words(self) -> int:
+        return (self.nb_k + 31) // 32
+
+    def as_c(self) -> BsaMask:
+        return BsaMask(self.bits.data_ptr(), self.counts.data_ptr(), self.row_offsets.data_ptr(),
+                       self.col_idx.data_ptr() if self.col_idx is not None else None,
+                       self.schedule.data_ptr(), self.B, self.H, self.nb_q, self.nb_k,
+                       self.words)
+
+
+def pack_mask(dense: torch.Tensor, with_lists: bool = True) -> PackedMask:
+    """dense uint8 [B, H, nb_q, nb_k] on the GPU -> PackedMask (bsa_pack_mask)."""
+    _require_cuda(dense, "dense", torch.uint8)
+    if dense.dim() != 4:
+        raise ValueError("dense must be [B, H, nb_q, nb_k]")
+    B, H, nb_q, nb_k = dense.shape
+    lib = _ffi.load()
+    dev = dense.device
+    words = (nb_k + 31) // 32
+    rows = B * H * nb_q
+    bits = torch.empty((B, H, nb_q, words), dtype=torch.int32, device=dev)
+    counts = torch.empty(rows, dtype=torch.int32, device=dev)
+    offsets = torch.empty(rows + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.empty(max(rows * nb_k, 1), dtype=torch.int32, device=dev) if with_lists else None
+    sched = torch.empty(rows, dtype=torch.int32, device=dev)
+    ws_bytes = lib.bsa_pack_mask_workspace(B, H, nb_q, nb_k)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    st = lib.bsa_pack_mask(dense.data_ptr(), B, H, nb_q, nb_k, bits.data_ptr(), counts.data_ptr(),
+                           offsets.data_ptr(), col_idx.data_ptr() if col_idx is not None else None,
+                           sched.data_ptr(), ws.data_ptr(), ws.numel(), _stream(dev))
+    _ffi.check(st, "bsa_pack_mask")
+    return PackedMask(bits, counts, offsets, col_idx, sched, B, H, nb_q, nb_k)
+
+
+def _grid_args(grid, tile):
+    T, Hs, Ws = (int(x) for x in grid)
+    tt, th, tw = (int(x) for x in tile)
+    return T, Hs, Ws, tt, th, tw
+
+
+def tile_permute(x: torch.Tensor, grid, tile, n_pad: int, out: torch.Tensor | None = None):
+    """[B, H, T*Hs*Ws, d] bf16 frame-major -> [B, H, n_pad, d] tile-major (bsa_tile_permute)."""
+    _require_cuda(x, "x", torch.bfloat16)
+    B, H, N, d = x.shape
+    T, Hs, Ws, tt, th, tw = _grid_args(grid, tile)
+    if N != T * Hs * Ws:
+        raise ValueError("token count does not match the grid")
+    if out is None:
+        out = torch.empty((B, H, n_pad, d), dtype=x.dtype, device=x.device)
+    _require_cuda(out, "out", torch.bfloat16)
+    st = _ffi.load().bsa_tile_permute(x.data_ptr(), out.data_ptr(), B, H, T, Hs, Ws, d, tt, th,
+                                      tw, n_pad, _stream(x.device))
+    _ffi.check(st, "bsa_tile_permute")
+    return out
+
+
+def tile_unpermute(y: torch.Tensor, grid, tile, out: torch.Tensor | None = None):
+    """[B, H, n_pad, d] bf16 tile-major -> [B, H, T*Hs*Ws, d] frame-major (bsa_tile_unpermute)."""
+    _require_cuda(y, "y", torch.bfloat16)
+    B, H, n_pad, d = y.shape
+    T, Hs, Ws, tt, th, tw = _grid_args(grid, tile)
+    if out is None:
+        out = torch.empty((B, H, T * Hs * Ws, d), dtype=y.dtype, device=y.device)
+    _require_cuda(out, "out", torch.bfloat16)
+    st = _ffi.load().bsa_tile_unpermute(y.data_ptr(), out.data_ptr(), B, H, T, Hs, Ws, d, tt, th,
+                                        tw, n_pad, _stream(y.device))
+    _ffi.check(st, "bsa_tile_unpermute")
+    return out
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask: PackedMask, n_valid: int,
+            block: int, softmax_scale: float | None = None, out: torch.Tensor | None = None,
+            lse: torch.Tensor | None = None):
+    """Block-sparse attention forward (bsa_forward) on tile-major q, k, v [B, H, n_pad, d] bf16.
+
+    Returns (out bf16 [B, H, n_pad, d], lse fp32 [B, H, n_pad])."""
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _require_cuda(t, name, torch.bfloat16)
+    B, H, n_pad, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v shapes differ")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, n_pad), dtype=torch.float32, device=q.device)
+    _require_cuda(out, "out", torch.bfloat16)
+    _require_cuda(lse, "lse", torch.float32)
+    cm = mask.as_c()
+    st = _ffi.load().bsa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(cm),
+                                 out.data_ptr(), lse.data_ptr(), B, H, int(n_valid), n_pad, d,
+                                 int(block), float(softmax_scale or 0.0), _stream(q.device))
+    _ffi.check(st, "bsa_forward")
+    return out, lse
+
+
+def device_error() -> int:
+    """Reads and clears the device error word (BSA_ERR_TIMEOUT after a barrier timeout)."""
+    code = ctypes.c_int(0)
+    _ffi.check(_ffi.load().bsa_get_device_error(ctypes.byref(code)), "bsa_get_device_error")
+    return code.value

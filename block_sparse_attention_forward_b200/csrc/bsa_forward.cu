@@ -1,0 +1,630 @@
+// bsa_forward.cu -- block-sparse attention forward for sm_100a.
+//
+// What it computes ("ScalingAttention", Sec. 4.3.2): the FlashAttention
+// forward whose dense key-block loop is replaced by the CRM forward iterator
+// of Appendix E (Algorithm 2), so only the kept key blocks of each query block
+// are visited; inside a kept tile the work is a dense tensor-core contraction,
+// across tiles an fp32 online softmax.
+//
+// How (B200-first, not the pages' Hopper design):
+//   * persistent grid, one CTA per SM, 192 threads in three roles:
+//       warps 0-3  softmax: one query row per thread (TMEM lane = row), online
+//                  max/sum in registers, P (bf16) written back into the S
+//                  columns of TMEM, O rescaled in TMEM, epilogue;
+//       warp  4    producer: walks the CRM words with the Algorithm 2 iterator
+//                  and issues TMA loads of Q, then K_j, V_j per kept block j
+//                  into a ring of shared-memory slots;
+//       warp  5    MMA issuer: tcgen05.mma S = Q K_j^T (both operands in
+//                  shared memory) into one of two TMEM S buffers, and
+//                  O += P V_j with P read straight from TMEM.
+//   * TMEM (512 columns): S0 at 0, S1 at 128, O at 256.  S(n+1) is computed
+//     while the softmax works on S(n).
+//   * work order: query tiles are taken from the count-descending schedule
+//     (heaviest first), CTA c handles tiles c, c + grid, ...
+//   * a tile is always 128 query rows; with 64-token blocks it holds two query
+//     blocks and walks the union of their CRM rows, each row masking the key
+//     blocks its own query block did not keep.
+//   * every barrier wait is bounded (about two seconds); a wait that runs out
+//     records BSA_ERR_TIMEOUT in a device word, the CTA drains what it has in
+//     flight and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "bsa.h"
+#include "bsa_internal.h"
+#include "sm100_ptx.cuh"
+
+__device__ int g_bsa_device_error = 0;
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kTileM = 128;  // query rows per tile = TMEM lanes
+constexpr int kThreads = 192;
+constexpr int kStages = 4;   // K/V ring slots
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+struct FwdParams {
+  const uint32_t* bits;     // [BH, nb, words]
+  const int32_t* schedule;  // [BH * nb] (used when one query block per tile)
+  __nv_bfloat16* out;       // [BH, n_pad, d]
+  float* lse;               // [BH, n_pad]
+  int BH, nb, words, n_valid, n_pad;
+  int num_tiles, tiles_per_head;
+  float scale_log2;
+};
+
+template <int D, int BLK>
+struct Cfg {
+  static constexpr int R = kTileM / BLK;                        // query blocks per tile
+  static constexpr int kRegions = D / 64;                       // 128-byte column groups
+  static constexpr uint32_t kQRegion = kTileM * 128;            // bytes per Q region
+  static constexpr uint32_t kQBytes = kRegions * kQRegion;
+  static constexpr uint32_t kKVRegion = BLK * 128;
+  static constexpr uint32_t kSlotBytes = kRegions * kKVRegion;  // one K or V tile
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffKV = kQBytes;
+  static constexpr uint32_t kOffBar = kOffKV + kStages * kSlotBytes;
+  // + barriers + alignment slack; at least 120 KB so that a second CTA never
+  // fits on the SM (each CTA owns all 512 TMEM columns)
+  static constexpr uint32_t kSmemUsed = kOffBar + 256 + 1024;
+  static constexpr uint32_t kSmemBytes = kSmemUsed > 120u * 1024u ? kSmemUsed : 120u * 1024u;
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, BLK, false);
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, true);
+};
+
+struct Barriers {
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_done[2];  // PV(k) completes on o_done[k & 1]
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Bounded wait: true when the phase of `parity` completed, false if this CTA
+// gave up (timeout here, or another role already aborted).
+__device__ __noinline__ bool wait_barrier(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > kTimeoutNs) {
+        *abort = 1;
+        atomicExch(&g_bsa_device_error, int(BSA_ERR_TIMEOUT));
+        return false;
+      }
+    }
+  }
+}
+
+// CRM forward iterator (Appendix E, Algorithm 2) over the OR of up to two CRM
+// rows: Init loads the first nonzero word, Next clears the lowest set bit and
+// skips empty words, Index is base + count-trailing-zeros or -1 at the end.
+struct CrmIter {
+  const uint32_t* row0;
+  const uint32_t* row1;
+  int w, words;
+  uint32_t val;
+  int base;
+  __device__ __forceinline__ void advance() {
+    while (val == 0u && w < words) {
+      val = __ldg(row0 + w) | (row1 ? __ldg(row1 + w) : 0u);
+      ++w;
+      base += 32;
+    }
+  }
+  __device__ __forceinline__ void init(const uint32_t* r0, const uint32_t* r1, int n_words) {
+    row0 = r0;
+    row1 = r1;
+    words = n_words;
+    w = 0;
+    val = 0u;
+    base = -32;
+    advance();
+  }
+  __device__ __forceinline__ void next() {
+    val &= val - 1u;
+    if (val == 0u) advance();
+  }
+  __device__ __forceinline__ int index() const { return val == 0u ? -1 : base + __ffs(val) - 1; }
+};
+
+struct TileInfo {
+  int bh, qb0;
+  const uint32_t* row0;
+  const uint32_t* row1;  // second query block's CRM row (two blocks per tile), or null
+};
+
+template <int R>
+__device__ __forceinline__ TileInfo tile_info(const FwdParams& p, int tile) {
+  TileInfo t;
+  if (R == 1) {
+    const int row = __ldg(p.schedule + tile);
+    t.bh = row / p.nb;
+    t.qb0 = row - t.bh * p.nb;
+  } else {
+    t.bh = tile / p.tiles_per_head;
+    t.qb0 = (tile - t.bh * p.tiles_per_head) * R;
+  }
+  t.row0 = p.bits + (int64_t(t.bh) * p.nb + t.qb0) * p.words;
+  t.row1 = (R > 1 && t.qb0 + 1 < p.nb) ? t.row0 + p.words : nullptr;
+  return t;
+}
+
+__device__ __forceinline__ int union_count(const TileInfo& t, int words) {
+  int c = 0;
+  for (int w = 0; w < words; ++w)
+    c += __popc(__ldg(t.row0 + w) | (t.row1 ? __ldg(t.row1 + w) : 0u));
+  return c;
+}
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(kThreads, 1)
+    bsa_forward_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = Cfg<D, BLK>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 128-byte swizzle atoms need 1024-byte aligned shared-memory tiles
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + C::kOffBar);
+  const uint32_t sQ = smem_addr(smem + C::kOffQ);
+  const uint32_t sKV = smem_addr(smem + C::kOffKV);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort = &bars->abort;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&bars->q_full), 1);
+    mbar_init(smem_addr(&bars->q_empty), 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_addr(&bars->kv_full[i]), 1);
+      mbar_init(smem_addr(&bars->kv_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_addr(&bars->s_full[i]), 1);
+      mbar_init(smem_addr(&bars->p_full[i]), kTileM);
+    }
+    mbar_init(smem_addr(&bars->o_done[0]), 1);
+    mbar_init(smem_addr(&bars->o_done[1]), 1);
+    mbar_init(smem_addr(&bars->drain), 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_addr(&bars->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t item = 0, q_iter = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        const TileInfo t = tile_info<C::R>(p, tile);
+        if (union_count(t, p.words) == 0) continue;
+        if (q_iter > 0 && !wait_barrier(smem_addr(&bars->q_empty), (q_iter - 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        const uint32_t qbar = smem_addr(&bars->q_full);
+        mbar_arrive_expect_tx(qbar, C::kQBytes);
+        const int32_t q_row = t.bh * p.n_pad + t.qb0 * BLK;
+#pragma unroll
+        for (int r = 0; r < C::kRegions; ++r)
+          tma_load_2d(sQ + r * C::kQRegion, &tm_q, qbar, r * 64, q_row);
+        ++q_iter;
+        CrmIter it;
+        it.init(t.row0, t.row1, p.words);
+        for (int j = it.index(); j >= 0; it.next(), j = it.index()) {
+          const int32_t kv_row = t.bh * p.n_pad + j * BLK;
+#pragma unroll
+          for (int kv = 0; kv < 2; ++kv) {  // K then V
+            const uint32_t slot = item % kStages;
+            if (item >= kStages &&
+                !wait_barrier(smem_addr(&bars->kv_empty[slot]), ((item / kStages) + 1) & 1,
+                              abort)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fbar = smem_addr(&bars->kv_full[slot]);
+            mbar_arrive_expect_tx(fbar, C::kSlotBytes);
+            const uint32_t dst = sKV + slot * C::kSlotBytes;
+#pragma unroll
+            for (int r = 0; r < C::kRegions; ++r)
+              tma_load_2d(dst + r * C::kKVRegion, kv == 0 ? &tm_k : &tm_v, fbar, r * 64, kv_row);
+            ++item;
+          }
+          if (!ok) break;
+        }
+      }
+      if (!ok) {
+        // let the copies already issued land before the CTA exits
+        const uint32_t first = item > kStages ? item - kStages : 0;
+        for (uint32_t i = first; i < item; ++i)
+          wait_barrier(smem_addr(&bars->kv_full[i % kStages]), (i / kStages) & 1, abort);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t item = 0, g = 0, q_iter = 0;
+      bool ok = true;
+      auto issue_pv = [&](uint32_t gi, uint32_t v_item, bool first) -> bool {
+        const uint32_t sb = gi & 1;
+        if (!wait_barrier(smem_addr(&bars->p_full[sb]), (gi >> 1) & 1, abort)) return false;
+        const uint32_t slot = v_item % kStages;
+        if (!wait_barrier(smem_addr(&bars->kv_full[slot]), (v_item / kStages) & 1, abort))
+          return false;
+        tc_fence_after();
+        const uint32_t p_tmem = tmem + (sb ? kTmemS1 : kTmemS0);
+        const uint32_t v_base = sKV + slot * C::kSlotBytes;
+#pragma unroll
+        for (int kk = 0; kk < BLK / 16; ++kk) {
+          // B = V tile, N (= head dim) contiguous: MN-major, 64-column groups
+          // C::kKVRegion apart (LBO), 8-key groups 1024 bytes apart (SBO)
+          const uint64_t bdesc = smem_desc_sw128(v_base + kk * 16 * 128, C::kKVRegion, 1024);
+          mma_ts(tmem + kTmemO, p_tmem + kk * 8, bdesc, C::kIdescPV, (first && kk == 0) ? 0u : 1u);
+        }
+        mma_commit(smem_addr(&bars->kv_empty[slot]));
+        mma_commit(smem_addr(&bars->o_done[gi & 1]));
+        return true;
+      };
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        const TileInfo t = tile_info<C::R>(p, tile);
+        const int cnt = union_count(t, p.words);
+        if (cnt == 0) continue;
+        if (!wait_barrier(smem_addr(&bars->q_full), q_iter & 1, abort)) {
+          ok = false;
+          break;
+        }
+        ++q_iter;
+        for (int n = 0; n < cnt; ++n) {
+          const uint32_t k_item = item + 2 * n;
+          const uint32_t slot = k_item % kStages;
+          if (!wait_barrier(smem_addr(&bars->kv_full[slot]), (k_item / kStages) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t s_tmem = tmem + (((g + n) & 1) ? kTmemS1 : kTmemS0);
+          const uint32_t k_base = sKV + slot * C::kSlotBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            // A = Q, B = K tile, both K-major; step 16 elements (32 bytes)
+            // inside a 128-byte swizzle atom, next atom group per 64 columns
+            const uint32_t off = (kk & 3) * 32;
+            const uint64_t adesc = smem_desc_sw128(sQ + (kk >> 2) * C::kQRegion + off, 16, 1024);
+            const uint64_t bdesc =
+                smem_desc_sw128(k_base + (kk >> 2) * C::kKVRegion + off, 16, 1024);
+            mma_ss(s_tmem, adesc, bdesc, C::kIdescS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(smem_addr(&bars->s_full[(g + n) & 1]));
+          mma_commit(smem_addr(&bars->kv_empty[slot]));
+          if (n == cnt - 1) mma_commit(smem_addr(&bars->q_empty));
+          if (n >= 1 && !issue_pv(g + n - 1, item + 2 * (n - 1) + 1, n - 1 == 0)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!ok) break;
+        if (!issue_pv(g + cnt - 1, item + 2 * (cnt - 1) + 1, cnt == 1)) {
+          ok = false;
+          break;
+        }
+        item += 2 * cnt;
+        g += cnt;
+      }
+      // drain: every MMA issued by this thread completes before TMEM is freed
+      mma_commit(smem_addr(&bars->drain));
+      wait_barrier(smem_addr(&bars->drain), 0, abort);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax (warps 0-3)
+    const int row = threadIdx.x;  // TMEM lane and query row inside the tile
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    uint32_t g = 0;
+    bool ok = true;
+    const bool has_tail = p.n_valid < p.n_pad;
+    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+      const TileInfo t = tile_info<C::R>(p, tile);
+      const int my_qb = t.qb0 + row / BLK;
+      const bool row_in_head = my_qb < p.nb;
+      const uint32_t* my_bits = p.bits + (int64_t(t.bh) * p.nb + my_qb) * p.words;
+      const int64_t tok = int64_t(t.qb0) * BLK + row;  // token index inside the head
+      float m_run = -INFINITY, l_run = 0.0f;
+
+      CrmIter it;
+      it.init(t.row0, t.row1, p.words);
+      int n = 0;
+      for (int j = it.index(); j >= 0; it.next(), j = it.index(), ++n) {
+        const uint32_t gi = g + n, sb = gi & 1;
+        // tcgen05.ld/st below are warp-collective: agree on the outcome first
+        if (!__all_sync(0xffffffffu, wait_barrier(smem_addr(&bars->s_full[sb]), (gi >> 1) & 1,
+                                                  abort))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t s_tmem = tmem + lane_base + (sb ? kTmemS1 : kTmemS0);
+        float s[BLK];
+#pragma unroll
+        for (int c0 = 0; c0 < BLK; c0 += 32) {
+          uint32_t r[32];
+          tmem_load32(s_tmem + c0, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[c0 + i] = __uint_as_float(r[i]);
+        }
+        bool member = row_in_head;
+        if (C::R > 1 && member) member = (__ldg(my_bits + (j >> 5)) >> (j & 31)) & 1u;
+        if (has_tail && j == p.nb - 1) {
+          const int valid = p.n_valid - j * BLK;
+#pragma unroll
+          for (int c = 0; c < BLK; ++c)
+            if (c >= valid) s[c] = -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BLK; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = member ? fmaxf(m_run, mx * p.scale_log2) : m_run;
+        const bool rescale = member && (m_run != -INFINITY) && (m_new > m_run);
+        const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O holds P(n-1) V(n-1) once that product has completed
+          if (!__all_sync(0xffffffffu,
+                          wait_barrier(smem_addr(&bars->o_done[(gi - 1) & 1]),
+                                       ((gi - 1) >> 1) & 1, abort))) {
+            ok = false;
+          } else {
+            tc_fence_after();
+            const uint32_t o_tmem = tmem + lane_base + kTmemO;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t r[32];
+              tmem_load32(o_tmem + c0, r);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+              tmem_store32(o_tmem + c0, r);
+            }
+          }
+        }
+        if (!ok) break;
+        float sum = 0.0f;
+        const float neg_m = -m_new;
+#pragma unroll
+        for (int c0 = 0; c0 < BLK; c0 += 64) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float p0 = 0.0f, p1 = 0.0f;
+            if (member) {
+              p0 = fast_exp2(fmaf(s[c0 + 2 * i], p.scale_log2, neg_m));
+              p1 = fast_exp2(fmaf(s[c0 + 2 * i + 1], p.scale_log2, neg_m));
+            }
+            sum += p0 + p1;
+            __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);  // low half = even key
+            pk[i] = *reinterpret_cast<uint32_t*>(&h);
+          }
+          // P overwrites the first half of this S buffer: packed bf16 pairs,
+          // 32 columns per 64 keys
+          tmem_store32(s_tmem + c0 / 2, pk);
+        }
+        if (member) {
+          l_run = l_run * alpha + sum;
+          m_run = m_new;
+        }
+        tmem_store_wait();
+        tc_fence_before();
+        mbar_arrive(smem_addr(&bars->p_full[sb]));
+      }
+      if (!ok) break;
+
+      // ---------------------------------------------------------- epilogue
+      const bool write_row = row_in_head;
+      const bool valid_row = tok < p.n_valid;
+      __nv_bfloat16* out_row = p.out + (int64_t(t.bh) * p.n_pad + tok) * D;
+      const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+      if (n > 0) {
+        if (!__all_sync(0xffffffffu,
+                        wait_barrier(smem_addr(&bars->o_done[(g + n - 1) & 1]),
+                                     ((g + n - 1) >> 1) & 1, abort))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t o_tmem = tmem + lane_base + kTmemO;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          tmem_load32(o_tmem + c0, r);
+          if (write_row) {
+            uint32_t pk[16];
+            const float sc = valid_row ? inv_l : 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * i]) * sc,
+                                                       __uint_as_float(r[2 * i + 1]) * sc);
+              pk[i] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(out_row + c0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      } else if (write_row) {
+        uint4* dst = reinterpret_cast<uint4*>(out_row);
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      if (write_row) {
+        float lse = -INFINITY;
+        if (valid_row && l_run > 0.0f) lse = (m_run + fast_log2(l_run)) * 0.69314718055994531f;
+        p.lse[int64_t(t.bh) * p.n_pad + tok] = lse;
+      }
+      g += n;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [rows, d] bf16 row-major, box = 64 columns x box_rows rows, 128-byte swizzle
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int d, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(d) * 2};
+  cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, int BLK>
+bsa_status launch_forward(const void* q, const void* k, const void* v, const bsa_mask* m,
+                          void* out, float* lse, int BH, int n_valid, int n_pad, float scale,
+                          cudaStream_t stream) {
+  using C = Cfg<D, BLK>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(bsa_forward_kernel<D, BLK>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(C::kSmemBytes)) != cudaSuccess)
+      return BSA_ERR_LAUNCH;
+    attr_set = true;
+  }
+  const int64_t rows = int64_t(BH) * n_pad;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, rows, D, kTileM) || !make_map(&tk, k, rows, D, BLK) ||
+      !make_map(&tv, v, rows, D, BLK))
+    return BSA_ERR_LAUNCH;
+  FwdParams p;
+  p.bits = m->bits;
+  p.schedule = m->schedule;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.BH = BH;
+  p.nb = n_pad / BLK;
+  p.words = (p.nb + 31) / 32;
+  p.n_valid = n_valid;
+  p.n_pad = n_pad;
+  p.tiles_per_head = (p.nb + C::R - 1) / C::R;
+  p.num_tiles = C::R == 1 ? BH * p.nb : BH * p.tiles_per_head;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int sms = bsa::num_sms();
+  if (sms <= 0) return BSA_ERR_LAUNCH;
+  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  bsa_forward_kernel<D, BLK><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  return bsa::launch_status();
+}
+
+}  // namespace
+
+extern "C" bsa_status bsa_forward(const void* q, const void* k, const void* v,
+                                  const bsa_mask* mask, void* out, float* lse, int B, int H,
+                                  int n_valid, int n_pad, int d, int block, float softmax_scale,
+                                  void* stream) {
+  if (!q || !k || !v || !mask || !out || !lse) return BSA_ERR_INVALID_ARG;
+  if (!mask->bits || !mask->schedule) return BSA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || n_pad <= 0 || n_valid <= 0 || block <= 0 || d <= 0)
+    return BSA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
+  if (block != 64 && block != 128) return BSA_ERR_UNSUPPORTED;
+  if (n_pad % block != 0) return BSA_ERR_UNSUPPORTED;
+  if (n_valid > n_pad || n_valid <= n_pad - block) return BSA_ERR_INVALID_ARG;
+  const int nb = n_pad / block;
+  if (mask->B != B || mask->H != H || mask->nb_q != nb || mask->nb_k != nb ||
+      mask->words != (nb + 31) / 32)
+    return BSA_ERR_INVALID_ARG;
+  if (int64_t(B) * H * n_pad >= (int64_t(1) << 31)) return BSA_ERR_OVERFLOW;
+  if (!bsa::aligned16(q) || !bsa::aligned16(k) || !bsa::aligned16(v) || !bsa::aligned16(out) ||
+      !bsa::aligned16(lse) || !bsa::aligned4(mask->bits) || !bsa::aligned4(mask->schedule))
+    return BSA_ERR_MISALIGNED;
+  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf(float(d));
+  const int BH = B * H;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128 && block == 128)
+    return launch_forward<128, 128>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
+  if (d == 128 && block == 64)
+    return launch_forward<128, 64>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
+  if (d == 64 && block == 128)
+    return launch_forward<64, 128>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
+  return launch_forward<64, 64>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
+}
+
+extern "C" bsa_status bsa_get_device_error(bsa_status* device_status) {
+  if (!device_status) return BSA_ERR_INVALID_ARG;
+  int host = 0, zero = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return BSA_ERR_LAUNCH;
+  if (cudaMemcpyFromSymbol(&host, g_bsa_device_error, sizeof(int)) != cudaSuccess)
+    return BSA_ERR_LAUNCH;
+  if (cudaMemcpyToSymbol(g_bsa_device_error, &zero, sizeof(int)) != cudaSuccess)
+    return BSA_ERR_LAUNCH;
+  *device_status = host == 0 ? BSA_OK : bsa_status(host);
+  return BSA_OK;
+}
+
+extern "C" int bsa_version(void) { return 100; }
+
+extern "C" const char* bsa_status_string(bsa_status s) {
+  switch (s) {
+    case BSA_OK: return "BSA_OK";
+    case BSA_ERR_INVALID_ARG: return "BSA_ERR_INVALID_ARG";
+    case BSA_ERR_UNSUPPORTED: return "BSA_ERR_UNSUPPORTED";
+    case BSA_ERR_MISALIGNED: return "BSA_ERR_MISALIGNED";
+    case BSA_ERR_OVERFLOW: return "BSA_ERR_OVERFLOW";
+    case BSA_ERR_LAUNCH: return "BSA_ERR_LAUNCH";
+    case BSA_ERR_TIMEOUT: return "BSA_ERR_TIMEOUT";
+    case BSA_ERR_WORKSPACE: return "BSA_ERR_WORKSPACE";
+  }
+  return "BSA_ERR_UNKNOWN";
+}

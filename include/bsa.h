@@ -1,0 +1,164 @@
+/*
+ * bsa.h -- C ABI of libbsa: bitmask-driven block-sparse attention forward for
+ * B200 (sm_100a).
+ *
+ * The operations follow "ScalingAttention: Discovering Intrinsic Sparse
+ * Attention Topology for Video Diffusion Transformers":
+ *   - Sec. 4.3.2 (CRM Kernel): a per-head block mask is encoded as one bitmask
+ *     row per query block (CRM), stored as aligned uint32 words, one bit per
+ *     key block; the kernel walks the active key blocks of a row with bit scan
+ *     and bit clear and runs the FlashAttention loop over them only.
+ *   - Appendix E (Algorithm 2): the CRM forward iterator (Init / Advance /
+ *     Next / Index).  Bit j of word w is key block 32*w + j.
+ *   - Sec. 5.4-5.5: token permutation that clusters tokens into hardware-
+ *     friendly blocks; here frame-major T x H x W tokens are gathered into
+ *     contiguous 3-D tiles so that one attention block is one tile.
+ *
+ * Conventions shared by every call:
+ *   - All data pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no device memory and frees nothing it did not create.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call is asynchronous on that stream; none synchronises.
+ *   - Arguments are checked on the host before any launch; a failed check
+ *     returns an error status and launches nothing.  No call throws, exits or
+ *     traps.  A launch failure returns BSA_ERR_LAUNCH.
+ *   - bf16 tensors are raw IEEE bfloat16 (2 bytes), row-major, with the shape
+ *     given beside each argument; the innermost index is contiguous.
+ *   - Every pointer passed to a data argument must be 16-byte aligned, else
+ *     BSA_ERR_MISALIGNED.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, inconsistent sizes */
+  BSA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. head dim 96) */
+  BSA_ERR_MISALIGNED = 3,  /* a data pointer is not 16-byte aligned */
+  BSA_ERR_OVERFLOW = 4,    /* an index or offset would not fit in int32 */
+  BSA_ERR_LAUNCH = 5,      /* the CUDA launch (or device query) failed */
+  BSA_ERR_TIMEOUT = 6,     /* a kernel gave up waiting on a pipeline barrier */
+  BSA_ERR_WORKSPACE = 7    /* workspace missing or smaller than required */
+} bsa_status;
+
+/* Device pointers produced by bsa_pack_mask and read by bsa_forward.  The
+ * struct itself lives in host memory. */
+typedef struct {
+  const uint32_t* bits;        /* [B, H, nb_q, words] CRM rows, words = (nb_k + 31) / 32 */
+  const int32_t* counts;       /* [B, H, nb_q] kept key blocks per query block */
+  const int32_t* row_offsets;  /* [B*H*nb_q + 1] exclusive prefix of counts */
+  const int32_t* col_idx;      /* [row_offsets[B*H*nb_q]] ascending kept key blocks per row */
+  const int32_t* schedule;     /* [B*H*nb_q] flat row ids, most kept blocks first, stable */
+  int B, H, nb_q, nb_k, words;
+} bsa_mask;
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int bsa_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* bsa_status_string(bsa_status status);
+
+/* ---------------------------------------------------------------------------
+ * bsa_pack_mask -- dense per-head block mask -> CRM rows + lists + schedule.
+ *
+ * Follows Sec. 4.3.2 (CRM representation: aligned uint32 rows, one bit per key
+ * block) with the bit order of Appendix E, Algorithm 2 (bit j of word w is key
+ * block 32*w + j; unused high bits of the last word are 0).
+ *
+ *   dense       [B, H, nb_q, nb_k] uint8; any nonzero byte marks a kept block.
+ *   bits        out [B, H, nb_q, words] uint32, words = (nb_k + 31) / 32.
+ *   counts      out [B*H*nb_q] int32, popcount of each row.
+ *   row_offsets out [B*H*nb_q + 1] int32, exclusive prefix sum of counts over
+ *               rows in (b, h, i) order; the last entry is the total.
+ *   col_idx     out, room for B*H*nb_q*nb_k int32 (the worst case); row r's
+ *               kept key blocks in ascending order at [row_offsets[r],
+ *               row_offsets[r+1]).  May be NULL to skip the lists.
+ *   schedule    out [B*H*nb_q] int32 flat row ids r = (b*H + h)*nb_q + i,
+ *               ordered by counts descending; equal counts keep ascending r.
+ *   workspace   device scratch of at least bsa_pack_mask_workspace(...) bytes,
+ *               16-byte aligned; its contents on entry do not matter.
+ *
+ * Alignment: dense needs no alignment; every other pointer must be 4-byte
+ * aligned (16-byte for workspace).  Errors: BSA_ERR_INVALID_ARG (null output,
+ * a size <= 0), BSA_ERR_OVERFLOW (B*H*nb_q*nb_k >= 2^31),
+ * BSA_ERR_WORKSPACE, BSA_ERR_LAUNCH.
+ * ------------------------------------------------------------------------- */
+size_t bsa_pack_mask_workspace(int B, int H, int nb_q, int nb_k);
+bsa_status bsa_pack_mask(const uint8_t* dense, int B, int H, int nb_q, int nb_k, uint32_t* bits,
+                         int32_t* counts, int32_t* row_offsets, int32_t* col_idx,
+                         int32_t* schedule, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* ---------------------------------------------------------------------------
+ * bsa_tile_permute / bsa_tile_unpermute -- 3-D tile gather (Sec. 5.4-5.5,
+ * token permutation into hardware-friendly blocks).
+ *
+ * Tokens of one (b, h) are frame-major: token (t, y, x) is at index
+ * (t*Hs + y)*Ws + x, N = T*Hs*Ws.  The tile-major order enumerates tiles
+ * (tile_t, tile_y, tile_x) row-major over a grid of tt x th x tw tiles; edge
+ * tiles are clipped to the grid (ragged) and their tokens concatenated with no
+ * holes; inside a tile tokens go (t, y, x) row-major.  Positions N..n_pad-1 are
+ * padding.
+ *
+ *   bsa_tile_permute:   in  [B, H, N, d] bf16 frame-major
+ *                       out [B, H, n_pad, d] bf16 tile-major, pad rows = 0.
+ *   bsa_tile_unpermute: in  [B, H, n_pad, d] bf16 tile-major
+ *                       out [B, H, N, d] bf16 frame-major (pad rows dropped).
+ *
+ * d must be a multiple of 8 (16-byte rows); n_pad >= N; in and out must not
+ * overlap.  Errors: BSA_ERR_INVALID_ARG, BSA_ERR_MISALIGNED, BSA_ERR_OVERFLOW
+ * (B*H*n_pad*d >= 2^40), BSA_ERR_LAUNCH.  Results are bit-exact copies.
+ * ------------------------------------------------------------------------- */
+bsa_status bsa_tile_permute(const void* in, void* out, int B, int H, int T, int Hs, int Ws, int d,
+                            int tt, int th, int tw, int n_pad, void* stream);
+bsa_status bsa_tile_unpermute(const void* in, void* out, int B, int H, int T, int Hs, int Ws,
+                              int d, int tt, int th, int tw, int n_pad, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * bsa_forward -- block-sparse attention forward (Sec. 4.3.2: the FlashAttention
+ * forward whose key-block loop is replaced by the CRM iterator of Appendix E,
+ * Algorithm 2; dense tensor-core work inside each kept tile).
+ *
+ * For each (b, h) and each valid query i < n_valid, with J the kept key blocks
+ * of query block i / block and keys j < n_valid:
+ *     s_j = scale * q_i . k_j   (j in a kept block; -inf otherwise)
+ *     out_i = sum_j softmax(s)_j v_j,   lse_i = max_j s_j + ln sum_j exp(s_j - max)
+ * Arithmetic: bf16 operands, fp32 accumulation and softmax, P rounded to bf16
+ * for the P.V product.  Query rows with no kept valid key, and pad rows
+ * i >= n_valid, get out = 0 and lse = -inf.
+ *
+ *   q, k, v  [B, H, n_pad, d] bf16 in tile-major order (see bsa_tile_permute).
+ *   mask     host pointer to a bsa_mask from bsa_pack_mask with the same B, H
+ *            and nb_q = nb_k = n_pad / block (bits and schedule are read).
+ *   out      [B, H, n_pad, d] bf16.
+ *   lse      [B, H, n_pad] fp32 (natural log, in units of the scaled logits).
+ *   softmax_scale <= 0 selects 1/sqrt(d).
+ *
+ * Supported: d in {64, 128}; block in {64, 128}; n_pad % block == 0;
+ * n_pad - block < n_valid <= n_pad.  Anything else: BSA_ERR_UNSUPPORTED or
+ * BSA_ERR_INVALID_ARG.  q, k, v, out and lse must be 16-byte aligned.
+ * A kernel that waits on a pipeline barrier for more than about two seconds
+ * gives up, records BSA_ERR_TIMEOUT for bsa_get_device_error and returns.
+ * ------------------------------------------------------------------------- */
+bsa_status bsa_forward(const void* q, const void* k, const void* v, const bsa_mask* mask,
+                       void* out, float* lse, int B, int H, int n_valid, int n_pad, int d,
+                       int block, float softmax_scale, void* stream);
+
+/* Reads and clears the device-side error word of the current device (set by a
+ * kernel that timed out on a barrier).  Synchronises the current device.
+ * Returns BSA_OK or BSA_ERR_TIMEOUT in *device_status; the return value is
+ * BSA_ERR_LAUNCH if the read itself failed. */
+bsa_status bsa_get_device_error(bsa_status* device_status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H_ */

@@ -1,0 +1,94 @@
+"""CPU-side checks of the C ABI: the library loads, exports every symbol that
+include/bsa.h declares, and rejects bad arguments on the host before any CUDA
+call (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "bsa.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bsa_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_attention_forward_b200 import _ffi, build
+    build.build()
+    return _ffi.load()
+
+
+def test_header_declarations_match_binding():
+    from block_sparse_attention_forward_b200 import _ffi
+    assert declared_functions() == sorted(_ffi.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    assert lib.bsa_status_string(0) == b"BSA_OK"
+    assert lib.bsa_status_string(6) == b"BSA_ERR_TIMEOUT"
+    assert lib.bsa_status_string(99) == b"BSA_ERR_UNKNOWN"
+    assert lib.bsa_version() >= 100
+
+
+def test_pack_mask_rejects_bad_args(lib):
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    # null output
+    assert lib.bsa_pack_mask(fake, 1, 1, 4, 4, None, fake, fake, fake, fake, fake, 4096, None) == 1
+    # non-positive size
+    assert lib.bsa_pack_mask(fake, 1, 0, 4, 4, fake, fake, fake, fake, fake, fake, 4096, None) == 1
+    # int32 overflow of B*H*nb_q*nb_k
+    assert lib.bsa_pack_mask(fake, 64, 64, 1024, 1024, fake, fake, fake, fake, fake, fake,
+                             1 << 30, None) == 4
+    # misaligned output
+    assert lib.bsa_pack_mask(fake, 1, 1, 4, 4, P(0x1001), fake, fake, fake, fake, fake, 4096,
+                             None) == 3
+    # workspace too small
+    assert lib.bsa_pack_mask_workspace(1, 1, 4, 4) > 0
+    assert lib.bsa_pack_mask(fake, 1, 1, 4, 4, fake, fake, fake, fake, fake, fake, 1, None) == 7
+
+
+def test_permute_rejects_bad_args(lib):
+    P = ctypes.c_void_p
+    a, b = P(0x1000), P(0x2000)
+    assert lib.bsa_tile_permute(None, b, 1, 1, 2, 2, 2, 8, 1, 1, 1, 8, None) == 1
+    assert lib.bsa_tile_permute(a, b, 1, 1, 2, 2, 2, 8, 1, 1, 1, 7, None) == 1  # n_pad < N
+    assert lib.bsa_tile_permute(a, b, 1, 1, 2, 2, 2, 6, 1, 1, 1, 8, None) == 2  # d % 8
+    assert lib.bsa_tile_permute(P(0x1008), b, 1, 1, 2, 2, 2, 8, 1, 1, 1, 8, None) == 3
+    assert lib.bsa_tile_unpermute(a, b, 1, 1, 2, 2, 0, 8, 1, 1, 1, 8, None) == 1
+
+
+def test_forward_rejects_bad_args(lib):
+    from block_sparse_attention_forward_b200._ffi import BsaMask
+    P = ctypes.c_void_p
+    a = P(0x10000)
+    m = BsaMask(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 1, 2, 8, 8, 1)
+    fwd = lib.bsa_forward
+    ok = dict(B=1, H=2, n_valid=1000, n_pad=1024, d=128, block=128)
+
+    def call(mask=m, q=a, out=a, **kw):
+        args = dict(ok)
+        args.update(kw)
+        return fwd(q, a, a, ctypes.byref(mask), out, a, args["B"], args["H"], args["n_valid"],
+                   args["n_pad"], args["d"], args["block"], 0.0, None)
+
+    assert call(q=None) == 1
+    assert call(d=96) == 2
+    assert call(block=32) == 2
+    assert call(n_pad=1000, n_valid=1000) == 2  # n_pad % block
+    assert call(n_valid=1025) == 1
+    assert call(n_valid=896) == 1  # a whole block of padding
+    bad = BsaMask(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 1, 2, 8, 8, 2)  # wrong words
+    assert call(mask=bad) == 1
+    assert call(out=P(0x10004)) == 3

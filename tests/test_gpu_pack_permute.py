@@ -1,0 +1,78 @@
+"""GPU parity of the integer steps against the oracle, bit-exact:
+CRM packing, kept-block lists, schedule (bsa_pack_mask) and the 3-D tile
+gather in both directions (bsa_tile_permute / bsa_tile_unpermute)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_forward_b200 import inputs as I
+from tests.helpers import bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def _pack_and_compare(dense: np.ndarray):
+    import block_sparse_attention_forward_b200 as bsa
+    B, H, nbq, nbk = dense.shape
+    pm = bsa.pack_mask(torch.from_numpy(dense).cuda())
+    torch.cuda.synchronize()
+    bits_ref = oracle.pack_bits(dense)
+    counts_ref, offsets_ref, col_ref = oracle.crm_lists(bits_ref)
+    sched_ref = oracle.schedule(counts_ref)
+    np.testing.assert_array_equal(pm.bits.cpu().numpy().view(np.uint32), bits_ref)
+    np.testing.assert_array_equal(pm.counts.cpu().numpy(), counts_ref)
+    np.testing.assert_array_equal(pm.row_offsets.cpu().numpy().astype(np.int64), offsets_ref)
+    total = int(offsets_ref[-1])
+    np.testing.assert_array_equal(pm.col_idx[:total].cpu().numpy(), col_ref)
+    np.testing.assert_array_equal(pm.schedule.cpu().numpy(), sched_ref)
+
+
+@pytest.mark.parametrize("name", ["tiny", "wan13b_480p", "wan14b_480p", "wan14b_720p"])
+def test_pack_mask_workloads(cuda_ok, name):
+    w = I.WORKLOADS[name]
+    _pack_and_compare(I.gen_mask(w))
+
+
+@pytest.mark.parametrize("shape,density", [((1, 1, 1, 1), 1.0), ((1, 3, 5, 33), 0.3),
+                                           ((2, 3, 64, 64), 0.0), ((1, 2, 100, 65), 0.9),
+                                           ((1, 4, 990, 990), 0.12), ((3, 1, 7, 1100), 0.5)])
+def test_pack_mask_edge_shapes(cuda_ok, shape, density):
+    rng = np.random.default_rng(sum(shape))
+    dense = (rng.random(shape) < density).astype(np.uint8)
+    dense[dense == 1] = rng.integers(1, 256, size=int(dense.sum()), dtype=np.uint8)
+    _pack_and_compare(dense)
+
+
+@pytest.mark.parametrize("name", ["tiny", "wan13b_480p", "wan14b_720p", "hunyuan_768p"])
+def test_permute_roundtrip_workload_grids(cuda_ok, name):
+    import block_sparse_attention_forward_b200 as bsa
+    w = I.WORKLOADS[name]
+    g = torch.Generator().manual_seed(w.seed)
+    x = torch.randn((1, 2, w.n, w.d), generator=g).to(torch.bfloat16)
+    grid, tile = (w.T, w.Hs, w.Ws), (w.tt, w.th, w.tw)
+    y = bsa.tile_permute(x.cuda(), grid, tile, w.n_pad)
+    z = bsa.tile_unpermute(y, grid, tile)
+    torch.cuda.synchronize()
+    perm = oracle.tile_order(w.T, w.Hs, w.Ws, w.tt, w.th, w.tw)
+    ref = oracle.permute(bf16_bits(x).reshape(2, w.n, w.d), perm, w.n_pad)
+    np.testing.assert_array_equal(bf16_bits(y).reshape(2, w.n_pad, w.d), ref)
+    np.testing.assert_array_equal(bf16_bits(z), bf16_bits(x))
+
+
+@pytest.mark.parametrize("grid,tile,d,n_extra", [((5, 7, 9), (2, 3, 4), 8, 3), ((1, 1, 1), (1, 1, 1), 64, 0),
+                                                 ((3, 17, 33), (2, 8, 16), 136, 100),
+                                                 ((4, 4, 4), (8, 8, 8), 128, 0)])
+def test_permute_ragged_shapes(cuda_ok, grid, tile, d, n_extra):
+    import block_sparse_attention_forward_b200 as bsa
+    n = grid[0] * grid[1] * grid[2]
+    n_pad = n + n_extra
+    g = torch.Generator().manual_seed(n)
+    x = torch.randn((2, 3, n, d), generator=g).to(torch.bfloat16)
+    y = bsa.tile_permute(x.cuda(), grid, tile, n_pad)
+    torch.cuda.synchronize()
+    perm = oracle.tile_order(*grid, *tile)
+    ref = oracle.permute(bf16_bits(x).reshape(6, n, d), perm, n_pad)
+    np.testing.assert_array_equal(bf16_bits(y).reshape(6, n_pad, d), ref)
+    z = bsa.tile_unpermute(y, grid, tile)
+    np.testing.assert_array_equal(bf16_bits(z), bf16_bits(x))
