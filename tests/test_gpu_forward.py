@@ -114,8 +114,8 @@ def test_forward_large_values_and_scale(cuda_ok):
     _, qo, ko, vo = oracle_inputs(w, q, k, v)
     ref_out, ref_lse = oracle.attention(qo, ko, vo, mask.reshape(BH, w.nb, w.nb), w.n, w.block,
                                         scale=0.3)
-    mx, mean, lse_err = compare_out(out_p.float().numpy().reshape(-1, w.d), ref_out,
-                                    lse.numpy().reshape(-1), ref_lse)
+    mx, mean, lse_err = compare_out(out_p.float().cpu().numpy().reshape(-1, w.d), ref_out,
+                                    lse.cpu().numpy().reshape(-1), ref_lse)
     assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS and lse_err <= LSE_ABS
 
 
