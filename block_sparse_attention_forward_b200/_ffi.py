@@ -28,6 +28,7 @@ EXPORTED = (
     "bsa_status_string",
     "bsa_pack_mask_workspace",
     "bsa_pack_mask",
+    "bsa_pack_mask_noalloc",
     "bsa_tile_permute",
     "bsa_tile_unpermute",
     "bsa_forward",
@@ -77,6 +78,8 @@ def load() -> ctypes.CDLL:
     lib.bsa_pack_mask_workspace.restype = SZ
     lib.bsa_pack_mask.argtypes = [P, I, I, I, I, P, P, P, P, P, P, SZ, P]
     lib.bsa_pack_mask.restype = I
+    lib.bsa_pack_mask_noalloc.argtypes = [P, I, I, I, I, P, P, P, P, P, P]
+    lib.bsa_pack_mask_noalloc.restype = I
     for name in ("bsa_tile_permute", "bsa_tile_unpermute"):
         fn = getattr(lib, name)
         fn.argtypes = [P, P, I, I, I, I, I, I, I, I, I, I, P]

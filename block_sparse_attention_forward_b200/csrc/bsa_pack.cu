@@ -17,6 +17,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "bsa.h"
 #include "bsa_internal.h"
 
@@ -209,6 +211,78 @@ extern "C" bsa_status bsa_pack_mask(const uint8_t* dense, int B, int H, int nb_q
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
   scan_sort_kernel<<<1, kSortThreads, 0, s>>>(counts, int(rows), nb_k, row_offsets, schedule,
                                                static_cast<int32_t*>(workspace));
+  if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
+  if (col_idx) {
+    write_lists_kernel<<<grid, 256, 0, s>>>(bits, rows, words, row_offsets, col_idx);
+    if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
+  }
+  return BSA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// bsa_pack_mask_noalloc: the same three kernels as bsa_pack_mask, with the
+// sort's scratch histogram in a fixed device array that this library owns,
+// for callers that cannot allocate device memory.
+//
+// The array below lives in every GPU's memory from the moment the library is
+// loaded on it until the process exits (512 KiB).  Host code cannot use the
+// symbol's name as a device address, so the device address is fetched once per
+// device with cudaGetSymbolAddress (with that device current) and cached.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kNoallocMaxNbK = 4095;  // key blocks per row the fixed scratch can sort
+constexpr int kNoallocScratchInts = kSortWarps * (kNoallocMaxNbK + 1);
+constexpr int kNoallocMaxDevices = 64;
+
+static __device__ __align__(256) int32_t g_pack_scratch[kNoallocScratchInts];
+
+std::mutex g_noalloc_mutex;
+int32_t* g_noalloc_scratch_ptr[kNoallocMaxDevices] = {};
+
+// Device address of g_pack_scratch on the current device (looked up on the
+// first call per device), or null if the lookup failed.
+int32_t* noalloc_scratch_for_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_pack_scratch) != cudaSuccess || !ptr) return nullptr;
+    g_noalloc_scratch_ptr[dev] = static_cast<int32_t*>(ptr);
+  }
+  return g_noalloc_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" bsa_status bsa_pack_mask_noalloc(const uint8_t* dense, int B, int H, int nb_q,
+                                            int nb_k, uint32_t* bits, int32_t* counts,
+                                            int32_t* row_offsets, int32_t* col_idx,
+                                            int32_t* schedule, void* stream) {
+  if (!dense || !bits || !counts || !row_offsets || !schedule) return BSA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || nb_q <= 0 || nb_k <= 0) return BSA_ERR_INVALID_ARG;
+  if (nb_k > kNoallocMaxNbK) return BSA_ERR_WORKSPACE;  // the fixed scratch is too small
+  const int64_t rows = int64_t(B) * H * nb_q;
+  if (rows * int64_t(nb_k) >= (int64_t(1) << 31)) return BSA_ERR_OVERFLOW;
+  if (!bsa::aligned4(bits) || !bsa::aligned4(counts) || !bsa::aligned4(row_offsets) ||
+      !bsa::aligned4(schedule) || (col_idx && !bsa::aligned4(col_idx)))
+    return BSA_ERR_MISALIGNED;
+  int32_t* scratch = noalloc_scratch_for_current_device();
+  if (!scratch) return BSA_ERR_LAUNCH;
+  const int sms = bsa::num_sms();
+  if (sms <= 0) return BSA_ERR_LAUNCH;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int words = (nb_k + 31) / 32;
+  const int64_t want_blocks = (rows + 7) / 8;  // 8 warps per block
+  const int grid = int(want_blocks < int64_t(sms) * 8 ? want_blocks : int64_t(sms) * 8);
+  pack_rows_kernel<<<grid, 256, 0, s>>>(dense, rows, nb_k, words, bits, counts);
+  if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
+  // scan_sort_kernel zeroes the histogram part of the scratch it uses before
+  // counting, so whatever an earlier call left there does not matter
+  scan_sort_kernel<<<1, kSortThreads, 0, s>>>(counts, int(rows), nb_k, row_offsets, schedule,
+                                               scratch);
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
   if (col_idx) {
     write_lists_kernel<<<grid, 256, 0, s>>>(bits, rows, words, row_offsets, col_idx);

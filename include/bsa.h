@@ -97,6 +97,31 @@ bsa_status bsa_pack_mask(const uint8_t* dense, int B, int H, int nb_q, int nb_k,
                          void* stream);
 
 /* ---------------------------------------------------------------------------
+ * bsa_pack_mask_noalloc -- bsa_pack_mask without a caller-supplied workspace.
+ *
+ * The paper has no counterpart: this variant exists for callers that cannot
+ * allocate device memory -- for example a plug-in host that hands a library
+ * only its input and output buffers, or a runtime that reserves all device
+ * memory up front and forbids later allocations (there cudaMalloc fails or
+ * stalls the device).  It computes exactly what bsa_pack_mask computes, with
+ * the same arguments minus the workspace, and allocates nothing: the sort's
+ * scratch is a fixed 512 KiB array inside the library, present on every GPU
+ * that loads it until the process exits.
+ *
+ * Limit: nb_k <= 4095; larger nb_k returns BSA_ERR_WORKSPACE (the built-in
+ * scratch is too small; use bsa_pack_mask).  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress) with that device
+ * current, so make that first call before any stream capture.  All calls share
+ * the one array: calls whose kernels overlap on a GPU (for example on two
+ * streams at once) race and give wrong results; calls in order on one stream
+ * are safe, since each call clears the scratch it uses.  Other errors as for
+ * bsa_pack_mask; BSA_ERR_LAUNCH also if the address lookup fails.
+ * ------------------------------------------------------------------------- */
+bsa_status bsa_pack_mask_noalloc(const uint8_t* dense, int B, int H, int nb_q, int nb_k,
+                                 uint32_t* bits, int32_t* counts, int32_t* row_offsets,
+                                 int32_t* col_idx, int32_t* schedule, void* stream);
+
+/* ---------------------------------------------------------------------------
  * bsa_tile_permute / bsa_tile_unpermute -- 3-D tile gather (Sec. 5.4-5.5,
  * token permutation into hardware-friendly blocks).
  *
