@@ -220,9 +220,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (smaller cases for profiling captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     w = I.WORKLOADS[args.workload]
+    if args.heads > 0:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
     if args.impl == "reference":
         return run_reference(args, w)
 

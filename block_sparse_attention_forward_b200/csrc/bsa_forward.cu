@@ -49,6 +49,7 @@ constexpr int kStages = 4;   // K/V ring slots
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
 
 struct FwdParams {
   const uint32_t* bits;     // [BH, nb, words]
@@ -367,27 +368,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t s_tmem = tmem + lane_base + (sb ? kTmemS1 : kTmemS0);
-        float s[BLK];
-#pragma unroll
-        for (int c0 = 0; c0 < BLK; c0 += 32) {
-          uint32_t r[32];
-          tmem_load32(s_tmem + c0, r);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c0 + i] = __uint_as_float(r[i]);
-        }
+        uint32_t sr[BLK];  // raw fp32 scores of this row, one tcgen05.ld
+        if constexpr (BLK == 128) tmem_load128(s_tmem, sr);
+        else tmem_load64(s_tmem, sr);
         bool member = row_in_head;
         if (C::R > 1 && member) member = (__ldg(my_bits + (j >> 5)) >> (j & 31)) & 1u;
         if (has_tail && j == p.nb - 1) {
           const int valid = p.n_valid - j * BLK;
 #pragma unroll
           for (int c = 0; c < BLK; ++c)
-            if (c >= valid) s[c] = -INFINITY;
+            if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < BLK; ++c) mx = fmaxf(mx, s[c]);
-        const float m_new = member ? fmaxf(m_run, mx * p.scale_log2) : m_run;
-        const bool rescale = member && (m_run != -INFINITY) && (m_new > m_run);
+        for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(sr[i]);
+#pragma unroll
+        for (int c = 8; c < BLK; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        // Lazy rescale: the reference max only moves when the row max grows by
+        // more than kRescaleLog2 (then O and l are scaled by alpha); otherwise
+        // p = exp2(s - m_ref) stays below 2^kRescaleLog2.  O / l is the same
+        // either way, since O and l always share one reference.
+        const float mx_scaled = mx * p.scale_log2;
+        bool rescale = false;
+        float m_new = m_run;
+        if (member) {
+          if (m_run == -INFINITY) {
+            m_new = mx_scaled;  // first kept block of this row: O and l are still 0
+          } else if (mx_scaled > m_run + kRescaleLog2) {
+            m_new = mx_scaled;
+            rescale = true;
+          }
+        }
         const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
         if (__any_sync(0xffffffffu, rescale)) {
           // O holds P(n-1) V(n-1) once that product has completed
@@ -409,26 +422,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        float sum = 0.0f;
+        float sum8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sum8[i] = 0.0f;
         const float neg_m = -m_new;
+        uint32_t pk[BLK / 2];
 #pragma unroll
-        for (int c0 = 0; c0 < BLK; c0 += 64) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float p0 = 0.0f, p1 = 0.0f;
-            if (member) {
-              p0 = fast_exp2(fmaf(s[c0 + 2 * i], p.scale_log2, neg_m));
-              p1 = fast_exp2(fmaf(s[c0 + 2 * i + 1], p.scale_log2, neg_m));
-            }
-            sum += p0 + p1;
-            __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);  // low half = even key
-            pk[i] = *reinterpret_cast<uint32_t*>(&h);
+        for (int i = 0; i < BLK / 2; ++i) {
+          float p0 = 0.0f, p1 = 0.0f;
+          if (member) {
+            p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), p.scale_log2, neg_m));
+            p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), p.scale_log2, neg_m));
           }
-          // P overwrites the first half of this S buffer: packed bf16 pairs,
-          // 32 columns per 64 keys
-          tmem_store32(s_tmem + c0 / 2, pk);
+          sum8[i & 7] += p0 + p1;
+          __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);  // low half = even key
+          pk[i] = *reinterpret_cast<uint32_t*>(&h);
         }
+        // P overwrites the first half of this S buffer: packed bf16 pairs, one
+        // 32-bit column per two keys
+        if constexpr (BLK == 128) tmem_store64(s_tmem, pk);
+        else tmem_store32(s_tmem, pk);
+        const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
+                          ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
         if (member) {
           l_run = l_run * alpha + sum;
           m_run = m_new;
