@@ -12,12 +12,15 @@
 //                  max/sum in registers, P (bf16) written back into the S
 //                  columns of TMEM, O rescaled in TMEM, epilogue;
 //       warp  4    producer: walks the CRM words with the Algorithm 2 iterator
-//                  and issues TMA loads of Q, then K_j, V_j per kept block j
-//                  into a ring of shared-memory slots;
-//       warp  5    MMA issuer: tcgen05.mma S = Q K_j^T (both operands in
-//                  shared memory) into one of two TMEM S buffers, and
-//                  O += P V_j with P read straight from TMEM.
-//   * TMEM (512 columns): S0 at 0, S1 at 128, O at 256.  S(n+1) is computed
+//                  and issues TMA loads of K_j, V_j per kept block j into a
+//                  ring of shared-memory slots;
+//       warp  5    MMA issuer: tcgen05.mma S = Q K_j^T into one of two TMEM S
+//                  buffers and O += P V_j.  Q and P are A operands read from
+//                  TMEM, so only K and V are read from shared memory (an M=128
+//                  N=128 product with both operands in shared memory would
+//                  need the whole 128 B/clk shared-memory port by itself).
+//   * TMEM (512 columns): S0 at 0, S1 at 128, O at 256, Q at 384 (bf16 pairs,
+//     written by the softmax threads once per tile).  S(n+1) is computed
 //     while the softmax works on S(n).
 //   * work order: query tiles are taken from the count-descending schedule
 //     (heaviest first), CTA c handles tiles c, c + grid, ...
@@ -45,13 +48,14 @@ using namespace sm100;
 
 constexpr int kTileM = 128;  // query rows per tile = TMEM lanes
 constexpr int kThreads = 192;
-constexpr int kStages = 4;   // K/V ring slots
+constexpr int kMaxStages = 8;  // K/V ring slots (as many as shared memory holds)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
+constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256, kTmemQ = 384;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
 
 struct FwdParams {
+  const __nv_bfloat16* q;   // [BH, n_pad, d]
   const uint32_t* bits;     // [BH, nb, words]
   const int32_t* schedule;  // [BH * nb] (used when one query block per tile)
   __nv_bfloat16* out;       // [BH, n_pad, d]
@@ -65,24 +69,25 @@ template <int D, int BLK>
 struct Cfg {
   static constexpr int R = kTileM / BLK;                        // query blocks per tile
   static constexpr int kRegions = D / 64;                       // 128-byte column groups
-  static constexpr uint32_t kQRegion = kTileM * 128;            // bytes per Q region
-  static constexpr uint32_t kQBytes = kRegions * kQRegion;
   static constexpr uint32_t kKVRegion = BLK * 128;
   static constexpr uint32_t kSlotBytes = kRegions * kKVRegion;  // one K or V tile
-  static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffKV = kQBytes;
+  static constexpr uint32_t kMaxSmem = 227u * 1024u;
+  static constexpr int kFitStages = int((kMaxSmem - 256 - 1024) / kSlotBytes);
+  static constexpr int kStages = kFitStages > kMaxStages ? kMaxStages : kFitStages;
+  static constexpr uint32_t kOffKV = 0;
   static constexpr uint32_t kOffBar = kOffKV + kStages * kSlotBytes;
   // + barriers + alignment slack; at least 120 KB so that a second CTA never
   // fits on the SM (each CTA owns all 512 TMEM columns)
   static constexpr uint32_t kSmemUsed = kOffBar + 256 + 1024;
   static constexpr uint32_t kSmemBytes = kSmemUsed > 120u * 1024u ? kSmemUsed : 120u * 1024u;
   static constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, BLK, false);
+  static_assert(kSmemUsed <= kMaxSmem, "shared memory budget");
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, true);
 };
 
 struct Barriers {
-  uint64_t q_full, q_empty;
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t q_full;  // the softmax threads have written this tile's Q into TMEM
+  uint64_t kv_full[kMaxStages], kv_empty[kMaxStages];
   uint64_t s_full[2], p_full[2];
   uint64_t o_done[2];  // PV(k) completes on o_done[k & 1]
   uint64_t drain;
@@ -90,10 +95,9 @@ struct Barriers {
   int abort;
 };
 
-// Bounded wait: true when the phase of `parity` completed, false if this CTA
-// gave up (timeout here, or another role already aborted).
-__device__ __noinline__ bool wait_barrier(uint32_t bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Bounded wait, slow path: spin until the phase of `parity` completed (true)
+// or this CTA gives up (timeout here, or another role already aborted).
+__device__ __noinline__ bool wait_barrier_slow(uint32_t bar, uint32_t parity, volatile int* abort) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -106,6 +110,13 @@ __device__ __noinline__ bool wait_barrier(uint32_t bar, uint32_t parity, volatil
       }
     }
   }
+}
+
+// Bounded wait: true when the phase of `parity` completed, false if this CTA
+// gave up.  Kept out of line: inlining it into the softmax loop measured slower.
+__device__ __noinline__ bool wait_barrier(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_barrier_slow(bar, parity, abort);
 }
 
 // CRM forward iterator (Appendix E, Algorithm 2) over the OR of up to two CRM
@@ -171,8 +182,7 @@ __device__ __forceinline__ int union_count(const TileInfo& t, int words) {
 
 template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads, 1)
-    bsa_forward_kernel(const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_k,
+    bsa_forward_kernel(const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = Cfg<D, BLK>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -180,15 +190,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   Barriers* bars = reinterpret_cast<Barriers*>(smem + C::kOffBar);
-  const uint32_t sQ = smem_addr(smem + C::kOffQ);
   const uint32_t sKV = smem_addr(smem + C::kOffKV);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &bars->abort;
 
   if (threadIdx.x == 0) {
-    mbar_init(smem_addr(&bars->q_full), 1);
-    mbar_init(smem_addr(&bars->q_empty), 1);
-    for (int i = 0; i < kStages; ++i) {
+    mbar_init(smem_addr(&bars->q_full), kTileM);
+    for (int i = 0; i < C::kStages; ++i) {
       mbar_init(smem_addr(&bars->kv_full[i]), 1);
       mbar_init(smem_addr(&bars->kv_empty[i]), 1);
     }
@@ -207,7 +215,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (warp == 4 && lane == 0) {
-    prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
   }
@@ -219,31 +226,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t item = 0, q_iter = 0;
+      uint32_t item = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         const TileInfo t = tile_info<C::R>(p, tile);
         if (union_count(t, p.words) == 0) continue;
-        if (q_iter > 0 && !wait_barrier(smem_addr(&bars->q_empty), (q_iter - 1) & 1, abort)) {
-          ok = false;
-          break;
-        }
-        const uint32_t qbar = smem_addr(&bars->q_full);
-        mbar_arrive_expect_tx(qbar, C::kQBytes);
-        const int32_t q_row = t.bh * p.n_pad + t.qb0 * BLK;
-#pragma unroll
-        for (int r = 0; r < C::kRegions; ++r)
-          tma_load_2d(sQ + r * C::kQRegion, &tm_q, qbar, r * 64, q_row);
-        ++q_iter;
         CrmIter it;
         it.init(t.row0, t.row1, p.words);
         for (int j = it.index(); j >= 0; it.next(), j = it.index()) {
           const int32_t kv_row = t.bh * p.n_pad + j * BLK;
 #pragma unroll
           for (int kv = 0; kv < 2; ++kv) {  // K then V
-            const uint32_t slot = item % kStages;
-            if (item >= kStages &&
-                !wait_barrier(smem_addr(&bars->kv_empty[slot]), ((item / kStages) + 1) & 1,
+            const uint32_t slot = item % C::kStages;
+            if (item >= C::kStages &&
+                !wait_barrier(smem_addr(&bars->kv_empty[slot]), ((item / C::kStages) + 1) & 1,
                               abort)) {
               ok = false;
               break;
@@ -261,9 +257,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         // let the copies already issued land before the CTA exits
-        const uint32_t first = item > kStages ? item - kStages : 0;
+        const uint32_t first = item > C::kStages ? item - C::kStages : 0;
         for (uint32_t i = first; i < item; ++i)
-          wait_barrier(smem_addr(&bars->kv_full[i % kStages]), (i / kStages) & 1, abort);
+          wait_barrier(smem_addr(&bars->kv_full[i % C::kStages]), (i / C::kStages) & 1, abort);
       }
     }
   } else if (warp == 5) {
@@ -274,16 +270,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_pv = [&](uint32_t gi, uint32_t v_item, bool first) -> bool {
         const uint32_t sb = gi & 1;
         if (!wait_barrier(smem_addr(&bars->p_full[sb]), (gi >> 1) & 1, abort)) return false;
-        const uint32_t slot = v_item % kStages;
-        if (!wait_barrier(smem_addr(&bars->kv_full[slot]), (v_item / kStages) & 1, abort))
+        const uint32_t slot = v_item % C::kStages;
+        if (!wait_barrier(smem_addr(&bars->kv_full[slot]), (v_item / C::kStages) & 1, abort))
           return false;
         tc_fence_after();
         const uint32_t p_tmem = tmem + (sb ? kTmemS1 : kTmemS0);
+        // B = V tile, N (= head dim) contiguous: MN-major, 64-column groups
+        // C::kKVRegion apart (LBO), 8-key groups 1024 bytes apart (SBO); 16
+        // keys (2048 bytes) per step
         const uint32_t v_base = sKV + slot * C::kSlotBytes;
 #pragma unroll
         for (int kk = 0; kk < BLK / 16; ++kk) {
-          // B = V tile, N (= head dim) contiguous: MN-major, 64-column groups
-          // C::kKVRegion apart (LBO), 8-key groups 1024 bytes apart (SBO)
           const uint64_t bdesc = smem_desc_sw128(v_base + kk * 16 * 128, C::kKVRegion, 1024);
           mma_ts(tmem + kTmemO, p_tmem + kk * 8, bdesc, C::kIdescPV, (first && kk == 0) ? 0u : 1u);
         }
@@ -302,27 +299,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++q_iter;
         for (int n = 0; n < cnt; ++n) {
           const uint32_t k_item = item + 2 * n;
-          const uint32_t slot = k_item % kStages;
-          if (!wait_barrier(smem_addr(&bars->kv_full[slot]), (k_item / kStages) & 1, abort)) {
+          const uint32_t slot = k_item % C::kStages;
+          if (!wait_barrier(smem_addr(&bars->kv_full[slot]), (k_item / C::kStages) & 1, abort)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t s_tmem = tmem + (((g + n) & 1) ? kTmemS1 : kTmemS0);
+          // A = Q from TMEM (16 elements = 8 columns per step); B = K tile,
+          // K-major: 16 elements (32 bytes) per step inside a 128-byte swizzle
+          // atom, the next 64-column group C::kKVRegion further
           const uint32_t k_base = sKV + slot * C::kSlotBytes;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            // A = Q, B = K tile, both K-major; step 16 elements (32 bytes)
-            // inside a 128-byte swizzle atom, next atom group per 64 columns
-            const uint32_t off = (kk & 3) * 32;
-            const uint64_t adesc = smem_desc_sw128(sQ + (kk >> 2) * C::kQRegion + off, 16, 1024);
             const uint64_t bdesc =
-                smem_desc_sw128(k_base + (kk >> 2) * C::kKVRegion + off, 16, 1024);
-            mma_ss(s_tmem, adesc, bdesc, C::kIdescS, kk > 0 ? 1u : 0u);
+                smem_desc_sw128(k_base + (kk >> 2) * C::kKVRegion + (kk & 3) * 32, 16, 1024);
+            mma_ts(s_tmem, tmem + kTmemQ + kk * 8, bdesc, C::kIdescS, kk > 0 ? 1u : 0u);
           }
           mma_commit(smem_addr(&bars->s_full[(g + n) & 1]));
           mma_commit(smem_addr(&bars->kv_empty[slot]));
-          if (n == cnt - 1) mma_commit(smem_addr(&bars->q_empty));
           if (n >= 1 && !issue_pv(g + n - 1, item + 2 * (n - 1) + 1, n - 1 == 0)) {
             ok = false;
             break;
@@ -354,6 +349,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t* my_bits = p.bits + (int64_t(t.bh) * p.nb + my_qb) * p.words;
       const int64_t tok = int64_t(t.qb0) * BLK + row;  // token index inside the head
       float m_run = -INFINITY, l_run = 0.0f;
+
+      if (union_count(t, p.words) > 0) {
+        // this row of Q -> TMEM lane `row`, bf16 pairs (low half = even
+        // element); every S product of the previous tile has completed (the
+        // last one was waited for), so its Q may be overwritten
+        uint32_t qr[D / 2];
+        if (row_in_head) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.q + (int64_t(t.bh) * p.n_pad + tok) * D);
+#pragma unroll
+          for (int i = 0; i < D / 8; ++i) {
+            const uint4 x = __ldg(src + i);
+            qr[4 * i] = x.x;
+            qr[4 * i + 1] = x.y;
+            qr[4 * i + 2] = x.z;
+            qr[4 * i + 3] = x.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < D / 2; ++i) qr[i] = 0u;
+        }
+        if constexpr (D == 128) tmem_store64(tmem + lane_base + kTmemQ, qr);
+        else tmem_store32(tmem + lane_base + kTmemQ, qr);
+        tmem_store_wait();
+        tc_fence_before();
+        mbar_arrive(smem_addr(&bars->q_full));
+      }
 
       CrmIter it;
       it.init(t.row0, t.row1, p.words);
@@ -558,11 +579,10 @@ bsa_status launch_forward(const void* q, const void* k, const void* v, const bsa
     attr_set = true;
   }
   const int64_t rows = int64_t(BH) * n_pad;
-  CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, rows, D, kTileM) || !make_map(&tk, k, rows, D, BLK) ||
-      !make_map(&tv, v, rows, D, BLK))
-    return BSA_ERR_LAUNCH;
+  CUtensorMap tk, tv;
+  if (!make_map(&tk, k, rows, D, BLK) || !make_map(&tv, v, rows, D, BLK)) return BSA_ERR_LAUNCH;
   FwdParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
   p.bits = m->bits;
   p.schedule = m->schedule;
   p.out = static_cast<__nv_bfloat16*>(out);
@@ -578,7 +598,7 @@ bsa_status launch_forward(const void* q, const void* k, const void* v, const bsa
   const int sms = bsa::num_sms();
   if (sms <= 0) return BSA_ERR_LAUNCH;
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-  bsa_forward_kernel<D, BLK><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  bsa_forward_kernel<D, BLK><<<grid, kThreads, C::kSmemBytes, stream>>>(tk, tv, p);
   return bsa::launch_status();
 }
 
