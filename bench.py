@@ -115,6 +115,30 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def forward_source_digest() -> str:
+    """sha256 over the forward kernel's sources (ties a DRAM capture to the code it measured)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("bsa_forward.cu", "sm100_ptx.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_attention_forward_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per forward launch from the committed ncu capture, or None when the
+    capture is missing, for another workload, or older than the kernel sources."""
+    path = os.path.join(ROOT, "profiles", "bsa_forward_dram.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("workload") != workload or rec.get("source_sha256") != forward_source_digest():
+        return None
+    return float(rec["dram_bytes_read"]) + float(rec["dram_bytes_write"])
+
+
 def gpu_selector(dev: torch.device) -> str:
     """nvidia-smi -i argument for this device (PCI bus id, else the CUDA index)."""
     try:
@@ -355,7 +379,8 @@ def main():
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
-                "frac": fwd_tflops / peak, "traffic": None, "kernel": "bsa_forward_kernel<128,128>",
+                "frac": fwd_tflops / peak, "traffic": recorded_traffic(w.name),
+                "kernel": "bsa_forward_kernel<128,128>",
                 "peak_source": f"{peak_src} bf16_tflops_sustained (dense bf16 cuBLAS, seconds-long loop)",
                 "fwd_ms": fwd_ms}
 
