@@ -19,6 +19,10 @@ Intrinsic Sparse Attention Topology for Video Diffusion Transformers"):
                          -- token reordering into 3-D tiles, Sec. 5.4 and 5.5.
 - ``attention``          -- Sec. 4.3.2 block-sparse FlashAttention forward,
                             written as plain masked softmax attention in fp64.
+- ``threshold_mask``     -- Sec. 4.1.2 (Eq. 2, M_p = 1(T <= p)) with one
+                            threshold per head (Algorithm 1, FAST).
+- ``threshold_resize``   -- Sec. 4.3.1, Eq. 7 (conservative bilinear resize of
+                            the threshold map with the ceiling rule).
 """
 from __future__ import annotations
 
@@ -69,6 +73,8 @@ def _load():
             lib.oracle_unpermute.argtypes = [P, P, I64, I64, I64, I, P]
             lib.oracle_attention.argtypes = [P, P, P, P, I64, I64, I64, I, I, ctypes.c_double,
                                              P, I64, I, P, P]
+            lib.oracle_threshold_mask.argtypes = [P, P, I, I, I, I, P]
+            lib.oracle_threshold_resize.argtypes = [P, I, I, I, P, I, I]
             _lib = lib
     return _lib
 
@@ -175,3 +181,24 @@ def attention(q_bits, k_bits, v_bits, mask, n_valid: int, block: int, scale: flo
                              n_pad, d, block, float(scale), rows_p, n_rows, int(dense_literal),
                              _ptr(out), _ptr(lse))
     return out, lse
+
+
+def threshold_mask(thr: np.ndarray, p: np.ndarray, B: int = 1) -> np.ndarray:
+    """thr float32 [H, nb_q, nb_k], p float32 [H] -> dense uint8 [B, H, nb_q, nb_k]."""
+    thr = np.ascontiguousarray(thr, dtype=np.float32)
+    p = np.ascontiguousarray(p, dtype=np.float32)
+    H, nb_q, nb_k = thr.shape
+    assert p.shape == (H,)
+    dense = np.zeros((B, H, nb_q, nb_k), dtype=np.uint8)
+    _load().oracle_threshold_mask(_ptr(thr), _ptr(p), B, H, nb_q, nb_k, _ptr(dense))
+    return dense
+
+
+def threshold_resize(src: np.ndarray, tq: int, tk: int) -> np.ndarray:
+    """src float32 [H, sq, sk] -> float32 [H, tq, tk] by Eq. 7 (min over the
+    source blocks with a nonzero bilinear weight at (u*sq/tq, v*sk/tk))."""
+    src = np.ascontiguousarray(src, dtype=np.float32)
+    H, sq, sk = src.shape
+    dst = np.empty((H, tq, tk), dtype=np.float32)
+    _load().oracle_threshold_resize(_ptr(src), H, sq, sk, _ptr(dst), int(tq), int(tk))
+    return dst

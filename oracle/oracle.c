@@ -277,3 +277,77 @@ void oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     free(qi);
   }
 }
+
+/* ------------------------------------------------------------------ */
+/* Threshold map -> block mask.                                        */
+/*                                                                     */
+/* ScalingAttention Sec. 4.1.2 (Eq. 2): T(u,v) is the smallest density */
+/* threshold at which block (u,v) joins the union of active regions,   */
+/* and a mask for any target density p is the comparison               */
+/* M_p = 1(T <= p).  Algorithm 1 (FAST, mask instantiation) picks one  */
+/* p* per layer, timestep and head, so here p holds one threshold per  */
+/* head and the map is shared by every batch item.                     */
+/*   thr   [H, nb_q, nb_k] float, p [H] float                          */
+/*   dense [B, H, nb_q, nb_k] uint8, 1 where thr <= p[h] (a NaN        */
+/*         threshold never compares true, so it is never kept)         */
+/* ------------------------------------------------------------------ */
+void oracle_threshold_mask(const float* thr, const float* p, int B, int H, int nb_q, int nb_k,
+                           uint8_t* dense) {
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int u = 0; u < nb_q; ++u)
+        for (int v = 0; v < nb_k; ++v) {
+          const float t = thr[((int64_t)h * nb_q + u) * nb_k + v];
+          const int64_t o = (((int64_t)b * H + h) * nb_q + u) * nb_k + v;
+          dense[o] = (t <= p[h]) ? 1 : 0;
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* Threshold map resize, ScalingAttention Sec. 4.3.1 (Eq. 7).          */
+/*                                                                     */
+/* Eq. 7 samples the base map by bilinear interpolation at             */
+/* (u / s_h, v / s_w) and applies a ceiling so that any overlap with   */
+/* an active region survives.  Reading: s_h = tq / sq and s_w = tk / sk */
+/* are the map's scale factors along its query and key axes, and the   */
+/* ceiling acts on the interpolated active-region indicator 1(T <= p): */
+/* the ceiling of a bilinear mix of 0/1 values is 1 exactly when some  */
+/* source block with a nonzero interpolation weight is active.  For    */
+/* every p at once that is the same as giving the target block the     */
+/* minimum threshold over those source blocks, which is what we store. */
+/* NaN thresholds (never active) are skipped; all-NaN gives NaN.       */
+/*   src [H, sq, sk] float  ->  dst [H, tq, tk] float                  */
+/* ------------------------------------------------------------------ */
+
+/* Source blocks with a nonzero bilinear weight at sample x = u / s,
+ * s = n_dst / n_src: floor(x) (weight 1 - frac, never 0) and floor(x) + 1
+ * (weight frac) when frac > 0, clamped to the last block. */
+static int bilinear_support(int u, int n_src, int n_dst, int* idx) {
+  const double x = (double)u * (double)n_src / (double)n_dst;
+  const double x0 = floor(x);
+  const double frac = x - x0;
+  int n = 0;
+  idx[n++] = (int)x0;
+  if (frac > 0.0) idx[n++] = ((int)x0 + 1 < n_src) ? (int)x0 + 1 : n_src - 1;
+  return n;
+}
+
+void oracle_threshold_resize(const float* src, int H, int sq, int sk, float* dst, int tq,
+                             int tk) {
+  for (int h = 0; h < H; ++h)
+    for (int u = 0; u < tq; ++u) {
+      int rows[2], cols[2];
+      const int nr = bilinear_support(u, sq, tq, rows);
+      for (int v = 0; v < tk; ++v) {
+        const int nc = bilinear_support(v, sk, tk, cols);
+        float m = NAN;
+        for (int a = 0; a < nr; ++a)
+          for (int c = 0; c < nc; ++c) {
+            const float t = src[((int64_t)h * sq + rows[a]) * sk + cols[c]];
+            if (isnan(t)) continue;
+            if (isnan(m) || t < m) m = t;
+          }
+        dst[((int64_t)h * tq + u) * tk + v] = m;
+      }
+    }
+}
