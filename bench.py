@@ -16,6 +16,10 @@ shape (different seed): the path shards by (batch, head) with no exchange, so
 there is no collective on the data path (weak scaling); the step time is the
 max over ranks.
 
+After the timed steps, `next_rows` reports the threshold-map steps measured
+on their own (L2 flushed before each call): bsa_pack_mask_from_threshold at the
+workload's block grid and bsa_threshold_resize of a 480p-grid map to it.
+
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of query blocks of the same workload (rank 0 only).
 """
@@ -226,6 +230,65 @@ def run_reference(args, w):
     return 0
 
 
+def time_device_us(fn, stream, flush: torch.Tensor, iters: int = 30, warmup: int = 10) -> float:
+    """Median device time in microseconds of fn() on `stream`, CUDA events around
+    each call, L2 flushed (a write larger than L2) before every call."""
+    for _ in range(warmup):
+        fn()
+    times = []
+    for _ in range(iters):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        times.append((e0, e1))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in times) * 1e3
+
+
+def measure_threshold_rows(w, dev, stream, hbm_gbs: float):
+    """Threshold-map rows: bsa_pack_mask_from_threshold at the workload's block grid
+    and bsa_threshold_resize of a map built at the 480p grid to this grid.  Both are
+    HBM-bound; algorithmic bytes = every input byte read once + every output byte
+    written once."""
+    import dataclasses
+
+    import block_sparse_attention_forward_b200 as bsa
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    thr, p = I.gen_threshold(w)
+    thr_d, p_d = torch.from_numpy(thr).to(dev), torch.from_numpy(p).to(dev)
+    pm = bsa.pack_mask_from_threshold(thr_d, p_d, B=w.B)
+    torch.cuda.synchronize(dev)
+    rows = w.B * w.H * w.nb
+    words = (w.nb + 31) // 32
+    kept = int(pm.row_offsets[-1])
+    pack_bytes = (thr.nbytes + p.nbytes + 4 * (rows * words + rows + rows + 1 + rows + kept))
+    pack_us = time_device_us(lambda: bsa.pack_mask_from_threshold(thr_d, p_d, B=w.B), stream,
+                             flush)
+    base_w = dataclasses.replace(I.WORKLOADS["wan14b_480p"], H=w.H)
+    base, _ = I.gen_threshold(base_w)
+    base_d = torch.from_numpy(base).to(dev)
+    dst = torch.empty((w.H, w.nb, w.nb), dtype=torch.float32, device=dev)
+    resize_bytes = base.nbytes + dst.numel() * 4
+    resize_us = time_device_us(lambda: bsa.threshold_resize(base_d, w.nb, w.nb, out=dst), stream,
+                               flush)
+    del flush
+
+    def entry(us, nbytes, **extra):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"us": us, "bytes": nbytes, "achieved_gbs": gbs, "frac_hbm": gbs / hbm_gbs,
+                "bound": "hbm", "l2": "flushed before each call", **extra}
+
+    return {
+        "pack_mask_from_threshold": entry(
+            pack_us, pack_bytes, launches=5, map=[w.H, w.nb, w.nb],
+            density=kept / (rows * w.nb)),
+        "threshold_resize": entry(resize_us, resize_bytes, launches=1,
+                                  src=[w.H, base_w.nb, base_w.nb], dst=[w.H, w.nb, w.nb]),
+    }
+
+
 def workload_config(w, mask):
     kept = I.kept_tiles(mask)
     total = w.B * w.H * w.nb * w.nb
@@ -244,6 +307,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip the threshold-map rows measured after the timed steps")
+    ap.add_argument("--only-next", action="store_true",
+                    help="measure only the threshold-map rows (a small case for profiling)")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (smaller cases for profiling captures)")
     args = ap.parse_args()
@@ -261,6 +328,15 @@ def main():
     world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.only_next:
+        peaks, _ = load_peaks()
+        rows = measure_threshold_rows(w, dev, torch.cuda.current_stream(dev),
+                                      float(peaks["hbm_gbs"]))
+        if rank == 0:
+            print(json.dumps({"workload": w.name, "next_rows": rows}), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return 0
     seed = w.seed + 7919 * rank
     q, k, v = I.gen_qkv(w, seed=seed)
     mask = I.gen_mask(w, q, k, seed=seed)
@@ -291,7 +367,7 @@ def main():
         bsa.tile_unpermute(out_p, grid, tile, out=out)
         return pm
 
-    launches_per_step = 3 + 3 + 1 + 1  # pack (3), permute q/k/v, forward, unpermute
+    launches_per_step = 5 + 3 + 1 + 1  # pack (5), permute q/k/v, forward, unpermute
 
     for _ in range(args.warmup):
         step(False)
@@ -376,6 +452,9 @@ def main():
 
     # ---------------------------------------------------------------- roofline
     peaks, peak_src = load_peaks()
+    next_rows = None
+    if not args.no_next:
+        next_rows = measure_threshold_rows(w, dev, stream, float(peaks["hbm_gbs"]))
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
@@ -403,6 +482,7 @@ def main():
             "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary(t_wall0, t_wall1),
             "peak_frac_step": value / peak,
+            "next_rows": next_rows,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

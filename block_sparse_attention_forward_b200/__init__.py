@@ -5,6 +5,7 @@ provides device memory and the current stream; each call checks dtypes,
 devices and contiguity, then passes raw pointers to the library.
 
     mask = pack_mask(dense_u8)                     # CRM rows, lists, schedule
+    mask = pack_mask_from_threshold(thr, p)        # or straight from a threshold map
     qp = tile_permute(q, grid, tile, n_pad)        # frame-major -> 3-D tiles
     out_p, lse = forward(qp, kp, vp, mask, n_valid, block)
     out = tile_unpermute(out_p, grid, tile)        # back to frame-major
@@ -19,8 +20,9 @@ import torch
 from . import _ffi
 from ._ffi import BsaError, BsaMask
 
-__all__ = ["BsaError", "PackedMask", "pack_mask", "tile_permute", "tile_unpermute", "forward",
-           "device_error", "version"]
+__all__ = ["BsaError", "PackedMask", "pack_mask", "pack_mask_from_threshold",
+           "threshold_resize", "tile_permute", "tile_unpermute", "forward", "device_error",
+           "version"]
 
 
 def _stream(device: torch.device) -> ctypes.c_void_p:
@@ -64,6 +66,22 @@ class PackedMask:
                        self.words)
 
 
+def _packed_outputs(B, H, nb_q, nb_k, dev, with_lists):
+    words = (nb_k + 31) // 32
+    rows = B * H * nb_q
+    return PackedMask(
+        torch.empty((B, H, nb_q, words), dtype=torch.int32, device=dev),
+        torch.empty(rows, dtype=torch.int32, device=dev),
+        torch.empty(rows + 1, dtype=torch.int32, device=dev),
+        torch.empty(max(rows * nb_k, 1), dtype=torch.int32, device=dev) if with_lists else None,
+        torch.empty(rows, dtype=torch.int32, device=dev), B, H, nb_q, nb_k)
+
+
+def _pack_pointers(pm: PackedMask):
+    return (pm.bits.data_ptr(), pm.counts.data_ptr(), pm.row_offsets.data_ptr(),
+            pm.col_idx.data_ptr() if pm.col_idx is not None else None, pm.schedule.data_ptr())
+
+
 def pack_mask(dense: torch.Tensor, with_lists: bool = True) -> PackedMask:
     """dense uint8 [B, H, nb_q, nb_k] on the GPU -> PackedMask (bsa_pack_mask)."""
     _require_cuda(dense, "dense", torch.uint8)
@@ -72,20 +90,56 @@ def pack_mask(dense: torch.Tensor, with_lists: bool = True) -> PackedMask:
     B, H, nb_q, nb_k = dense.shape
     lib = _ffi.load()
     dev = dense.device
-    words = (nb_k + 31) // 32
-    rows = B * H * nb_q
-    bits = torch.empty((B, H, nb_q, words), dtype=torch.int32, device=dev)
-    counts = torch.empty(rows, dtype=torch.int32, device=dev)
-    offsets = torch.empty(rows + 1, dtype=torch.int32, device=dev)
-    col_idx = torch.empty(max(rows * nb_k, 1), dtype=torch.int32, device=dev) if with_lists else None
-    sched = torch.empty(rows, dtype=torch.int32, device=dev)
+    pm = _packed_outputs(B, H, nb_q, nb_k, dev, with_lists)
     ws_bytes = lib.bsa_pack_mask_workspace(B, H, nb_q, nb_k)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    st = lib.bsa_pack_mask(dense.data_ptr(), B, H, nb_q, nb_k, bits.data_ptr(), counts.data_ptr(),
-                           offsets.data_ptr(), col_idx.data_ptr() if col_idx is not None else None,
-                           sched.data_ptr(), ws.data_ptr(), ws.numel(), _stream(dev))
+    st = lib.bsa_pack_mask(dense.data_ptr(), B, H, nb_q, nb_k, *_pack_pointers(pm),
+                           ws.data_ptr(), ws.numel(), _stream(dev))
     _ffi.check(st, "bsa_pack_mask")
-    return PackedMask(bits, counts, offsets, col_idx, sched, B, H, nb_q, nb_k)
+    return pm
+
+
+def pack_mask_from_threshold(thr: torch.Tensor, p: torch.Tensor, B: int = 1,
+                             with_lists: bool = True) -> PackedMask:
+    """Threshold map fp32 [H, nb_q, nb_k] and per-head thresholds fp32 [H], both on
+    the GPU -> PackedMask of M_p = 1(thr <= p[h]) for B batch items
+    (bsa_pack_mask_from_threshold)."""
+    _require_cuda(thr, "thr", torch.float32)
+    _require_cuda(p, "p", torch.float32)
+    if thr.dim() != 3:
+        raise ValueError("thr must be [H, nb_q, nb_k]")
+    H, nb_q, nb_k = thr.shape
+    if p.shape != (H,):
+        raise ValueError("p must be [H]")
+    lib = _ffi.load()
+    dev = thr.device
+    pm = _packed_outputs(int(B), H, nb_q, nb_k, dev, with_lists)
+    ws_bytes = lib.bsa_pack_mask_workspace(int(B), H, nb_q, nb_k)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    st = lib.bsa_pack_mask_from_threshold(thr.data_ptr(), p.data_ptr(), int(B), H, nb_q, nb_k,
+                                          *_pack_pointers(pm), ws.data_ptr(), ws.numel(),
+                                          _stream(dev))
+    _ffi.check(st, "bsa_pack_mask_from_threshold")
+    return pm
+
+
+def threshold_resize(src: torch.Tensor, tq: int, tk: int,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    """Threshold map fp32 [H, sq, sk] on the GPU -> fp32 [H, tq, tk] by the
+    conservative resize of Eq. 7 (bsa_threshold_resize)."""
+    _require_cuda(src, "src", torch.float32)
+    if src.dim() != 3:
+        raise ValueError("src must be [H, sq, sk]")
+    H, sq, sk = src.shape
+    if out is None:
+        out = torch.empty((H, int(tq), int(tk)), dtype=torch.float32, device=src.device)
+    _require_cuda(out, "out", torch.float32)
+    if out.shape != (H, tq, tk):
+        raise ValueError("out must be [H, tq, tk]")
+    st = _ffi.load().bsa_threshold_resize(src.data_ptr(), H, sq, sk, out.data_ptr(), int(tq),
+                                          int(tk), _stream(src.device))
+    _ffi.check(st, "bsa_threshold_resize")
+    return out
 
 
 def _grid_args(grid, tile):

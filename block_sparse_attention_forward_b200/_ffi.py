@@ -29,6 +29,8 @@ EXPORTED = (
     "bsa_pack_mask_workspace",
     "bsa_pack_mask",
     "bsa_pack_mask_noalloc",
+    "bsa_pack_mask_from_threshold",
+    "bsa_threshold_resize",
     "bsa_tile_permute",
     "bsa_tile_unpermute",
     "bsa_forward",
@@ -80,6 +82,10 @@ def load() -> ctypes.CDLL:
     lib.bsa_pack_mask.restype = I
     lib.bsa_pack_mask_noalloc.argtypes = [P, I, I, I, I, P, P, P, P, P, P]
     lib.bsa_pack_mask_noalloc.restype = I
+    lib.bsa_pack_mask_from_threshold.argtypes = [P, P, I, I, I, I, P, P, P, P, P, P, SZ, P]
+    lib.bsa_pack_mask_from_threshold.restype = I
+    lib.bsa_threshold_resize.argtypes = [P, I, I, I, P, I, I, P]
+    lib.bsa_threshold_resize.restype = I
     for name in ("bsa_tile_permute", "bsa_tile_unpermute"):
         fn = getattr(lib, name)
         fn.argtypes = [P, P, I, I, I, I, I, I, I, I, I, I, P]

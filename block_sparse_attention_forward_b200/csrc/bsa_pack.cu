@@ -1,19 +1,30 @@
-// bsa_pack.cu -- dense per-head block masks -> CRM rows, counts, row offsets,
+// bsa_pack.cu -- per-head block masks -> CRM rows, counts, row offsets,
 // ascending key-block lists and the count-ordered schedule.
 //
 // CRM layout ("ScalingAttention", Sec. 4.3.2 and Appendix E, Algorithm 2): one
 // row of uint32 words per query block; bit j of word w is key block 32*w + j
 // (the iterator's base grows by 32 per word and the index is base + CTZ).
 //
-// Three launches on the caller's stream:
-//   1. pack_rows:   one warp per row; a coalesced 32-byte read of the dense row
-//                   per word, __ballot_sync builds the word, popcounts sum.
-//   2. scan_sort:   one CTA; exclusive prefix of counts -> row_offsets, and a
-//                   stable counting sort of rows by count (descending) with
-//                   per-warp histograms kept in the caller's workspace.
-//   3. write_lists: one warp per row; each lane takes one word, a warp scan of
-//                   popcounts gives its output offset, set bits are written in
-//                   ascending order.
+// Five launches on the caller's stream:
+//   1. rows:        one warp per row; a coalesced read of the row per word,
+//                   __ballot_sync builds the word, popcounts sum.  Two
+//                   variants: a dense uint8 mask (bsa_pack_mask), or a
+//                   per-head threshold map with one threshold per head,
+//                   keeping block (u, v) when T(u, v) <= p_h (Sec. 4.1.2,
+//                   M_p = 1(T <= p); Algorithm 1 picks p per layer, timestep
+//                   and head; bsa_pack_mask_from_threshold).
+//   2. tile_hist:   rows are cut into tiles of kTileRows; one CTA per tile
+//                   histograms its counts in shared memory and sums them.
+//   3. tile_scan:   one CTA; exclusive scan of the tile sums (row bases), and
+//                   of the histograms in (count descending, tile ascending)
+//                   order, which gives every (tile, count) its first slot in
+//                   the schedule.
+//   4. tile_place:  one CTA per tile; row_offsets from a block scan, then the
+//                   tile's warps take turns placing their rows at their
+//                   count's next slot -- in row order, so the sort is stable.
+//   5. write_lists: one warp per row; words are taken one at a time and each
+//                   lane writes its key block at the row's running offset, so
+//                   each store instruction writes consecutive addresses.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -24,49 +35,110 @@
 
 namespace {
 
-constexpr int kSortThreads = 1024;
-constexpr int kSortWarps = kSortThreads / 32;
+constexpr int kRowWarps = 8;  // warps (rows) per block of the row-parallel launches
+
+// One row per warp.  `kept(j)` tells whether key block j (< nb_k) is kept.
+// Words are built 32 at a time: for word k of the group every lane tests its
+// key block and a ballot forms the word, which lane k keeps; the group is then
+// stored with one coalesced write.  Loads of a partly filled last word are
+// clamped to the row, and lanes past its end vote false.  (Unrolled by 8 at 32
+// registers: measured faster than issuing all of a group's loads up front at
+// 58-63 registers, where fewer warps fit on an SM.)
+template <typename Kept>
+__device__ __forceinline__ void pack_one_row(const Kept kept, int nb_k, int words,
+                                             uint32_t* __restrict__ out, int32_t* count) {
+  const int lane = threadIdx.x & 31;
+  int total = 0;
+  for (int w0 = 0; w0 < words; w0 += 32) {
+    const int n = min(32, words - w0);
+    uint32_t mine = 0;
+#pragma unroll 8
+    for (int k = 0; k < n; ++k) {
+      const int j = (w0 + k) * 32 + lane;
+      const bool keep = kept(min(j, nb_k - 1)) & (j < nb_k);
+      const uint32_t word = __ballot_sync(0xffffffffu, keep);
+      mine = lane == k ? word : mine;
+    }
+    if (lane < n) out[w0 + lane] = mine;
+    total += __popc(mine);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+  if (lane == 0) *count = total;
+}
+
+// Row tests, passed by value so their state stays in registers.
+struct DenseKept {
+  const uint8_t* row;
+  __device__ __forceinline__ bool operator()(int j) const { return __ldg(row + j) != 0; }
+};
+struct ThresholdKept {
+  const float* row;
+  float p;
+  __device__ __forceinline__ bool operator()(int j) const { return __ldg(row + j) <= p; }
+};
 
 __global__ void __launch_bounds__(256) pack_rows_kernel(const uint8_t* __restrict__ dense,
-                                                        int64_t rows, int nb_k, int words,
+                                                        int rows, int nb_k, int words,
                                                         uint32_t* __restrict__ bits,
                                                         int32_t* __restrict__ counts) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t n_warps = (int64_t(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t r = warp; r < rows; r += n_warps) {
-    const uint8_t* row = dense + r * nb_k;
-    uint32_t* out = bits + r * words;
-    int total = 0;
-    for (int w = 0; w < words; ++w) {
-      const int j = w * 32 + lane;
-      const bool kept = (j < nb_k) && (row[j] != 0);
-      const uint32_t word = __ballot_sync(0xffffffffu, kept);
-      if (lane == 0) out[w] = word;
-      total += __popc(word);
-    }
-    if (lane == 0) counts[r] = total;
+  const int n_warps = gridDim.x * kRowWarps;
+  for (int r = blockIdx.x * kRowWarps + (threadIdx.x >> 5); r < rows; r += n_warps) {
+    const uint8_t* row = dense + size_t(r) * nb_k;
+    pack_one_row(DenseKept{row}, nb_k, words, bits + size_t(r) * words, counts + r);
   }
 }
 
-// Block-wide exclusive scan of one value per thread; returns the prefix and
-// writes the block total to *total.  `smem` holds kSortWarps ints.
+// Threshold rows: row r = (b, h, u) reads map row (h, u), the same for every
+// batch item (map_rows = H * nb_q).  A NaN threshold compares false: never kept.
+__global__ void __launch_bounds__(256)
+    pack_threshold_rows_kernel(const float* __restrict__ thr, const float* __restrict__ p,
+                               int nb_q, int map_rows, int rows, int nb_k, int words,
+                               uint32_t* __restrict__ bits, int32_t* __restrict__ counts) {
+  const int n_warps = gridDim.x * kRowWarps;
+  for (int r = blockIdx.x * kRowWarps + (threadIdx.x >> 5); r < rows; r += n_warps) {
+    const int hu = r % map_rows;
+    const float p_h = __ldg(p + hu / nb_q);
+    const float* row = thr + size_t(hu) * nb_k;
+    pack_one_row(ThresholdKept{row, p_h}, nb_k, words, bits + size_t(r) * words, counts + r);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Offsets and the stable count-descending schedule, over tiles of kTileRows
+// rows (one thread per row in the tile launches).  The histograms are kept
+// "count descending major": entry (d, t) with d = nb_k - count is at
+// d * tiles + t, so that one contiguous exclusive scan gives every (count,
+// tile) pair its first slot in the schedule.
+// ---------------------------------------------------------------------------
+constexpr int kTileRows = 1024;
+constexpr int kTileWarps = kTileRows / 32;
+constexpr int kScanRun = 8;  // values per thread in one pass of a chunked scan
+// Dynamic shared memory any sort launch asks for, and so the largest per-count
+// table a tile keeps there: nb_k + 1 ints.
+constexpr size_t kMaxDynamicSmem = 196608;
+constexpr int kMaxBins = int(kMaxDynamicSmem / sizeof(int32_t));
+
+// Block-wide exclusive scan of one value per thread (kTileRows threads);
+// returns the prefix and writes the block total to *total.  `smem` holds 33
+// ints.  Starts and ends with a barrier's worth of ordering: shared-memory
+// writes made before the call are visible to every thread after it.
 __device__ __forceinline__ int block_exclusive_scan(int x, int* smem, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = x;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, incl, o);
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += y;
   }
   if (lane == 31) smem[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int v = smem[lane];
+    const int v = smem[lane];
     int vi = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, vi, o);
+      const int y = __shfl_up_sync(0xffffffffu, vi, o);
       if (lane >= o) vi += y;
     }
     smem[lane] = vi - v;  // exclusive prefix of warp totals
@@ -79,110 +151,262 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* smem, int* total
   return result;
 }
 
-// hist: kSortWarps * (nb_k + 1) ints of workspace, laid out [count desc][warp]
-// so that one flat exclusive scan yields every (warp, count) output base.
-__global__ void __launch_bounds__(kSortThreads, 1)
-    scan_sort_kernel(const int32_t* __restrict__ counts, int rows, int nb_k,
-                     int32_t* __restrict__ row_offsets, int32_t* __restrict__ schedule,
-                     int32_t* __restrict__ hist) {
-  __shared__ int scan_smem[33];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int n_bins = nb_k + 1;
-  const int hist_len = kSortWarps * n_bins;
+// In-place exclusive scan of a[0..n) by one CTA of kTileRows threads, in
+// chunks of kScanChunk values staged through shared memory `buf` (coalesced
+// global reads and writes; each thread scans a contiguous run of kScanRun
+// values of the chunk).  Rows of 32 values are padded by one word so that the
+// runs of a warp fall in distinct banks.  Returns the total.
+constexpr int kScanChunk = kTileRows * kScanRun;
+constexpr int kScanBufInts = kScanChunk + kScanChunk / 32;
+__device__ __forceinline__ int padded(int i) { return i + (i >> 5); }
 
-  // 1. row_offsets = exclusive prefix of counts
+__device__ __forceinline__ int cta_exclusive_scan_inplace(int32_t* a, int n, int* smem,
+                                                          int* buf) {
   int carry = 0;
-  for (int base = 0; base < rows; base += kSortThreads) {
-    const int r = base + tid;
-    const int c = r < rows ? counts[r] : 0;
-    int chunk_total;
-    const int pre = block_exclusive_scan(c, scan_smem, &chunk_total);
-    if (r < rows) row_offsets[r] = carry + pre;
-    carry += chunk_total;
-  }
-  if (tid == 0) row_offsets[rows] = carry;
-
-  // 2. per-warp histograms of counts over contiguous row segments
-  // the histogram is touched through L2 only (atomics, __ldcg/__stcg)
-  for (int i = tid; i < hist_len; i += kSortThreads) __stcg(hist + i, 0);
-  __syncthreads();
-  const int seg = (rows + kSortWarps - 1) / kSortWarps;
-  const int seg_lo = min(rows, warp * seg), seg_hi = min(rows, seg_lo + seg);
-  for (int r = seg_lo + lane; r < seg_hi; r += 32) {
-    const int c = counts[r];
-    atomicAdd(&hist[(nb_k - c) * kSortWarps + warp], 1);
-  }
-  __syncthreads();
-
-  // 3. exclusive scan of hist in (count descending, warp ascending) order
-  carry = 0;
-  for (int base = 0; base < hist_len; base += kSortThreads) {
-    const int i = base + tid;
-    const int h = i < hist_len ? __ldcg(hist + i) : 0;
-    int chunk_total;
-    const int pre = block_exclusive_scan(h, scan_smem, &chunk_total);
-    if (i < hist_len) __stcg(hist + i, carry + pre);
-    carry += chunk_total;
-  }
-  __syncthreads();
-
-  // 4. stable placement: each warp walks its segment in row order
-  for (int base = seg_lo; base < seg_hi; base += 32) {
-    const int r = base + lane;
-    const bool active = r < seg_hi;
-    const unsigned act = __ballot_sync(0xffffffffu, active);
-    if (active) {
-      const int c = counts[r];
-      const unsigned peers = __match_any_sync(act, c);
-      const int rank = __popc(peers & ((1u << lane) - 1u));
-      int* slot = &hist[(nb_k - c) * kSortWarps + warp];
-      const int pos = __ldcg(slot) + rank;
-      schedule[pos] = r;
-      __syncwarp(act);
-      if (rank == 0) __stcg(slot, pos + __popc(peers));
+  for (int base = 0; base < n; base += kScanChunk) {
+    const int m = min(kScanChunk, n - base);
+    for (int i = threadIdx.x; i < kScanChunk; i += kTileRows)
+      buf[padded(i)] = i < m ? a[base + i] : 0;
+    __syncthreads();
+    const int i0 = threadIdx.x * kScanRun;
+    int v[kScanRun];
+    int run = 0;
+#pragma unroll
+    for (int k = 0; k < kScanRun; ++k) {
+      v[k] = buf[padded(i0 + k)];
+      run += v[k];
     }
-    __syncwarp();
+    int chunk_total;
+    int pre = carry + block_exclusive_scan(run, smem, &chunk_total);
+#pragma unroll
+    for (int k = 0; k < kScanRun; ++k) {
+      buf[padded(i0 + k)] = pre;
+      pre += v[k];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < m; i += kTileRows) a[base + i] = buf[padded(i)];
+    __syncthreads();  // the next chunk reuses buf
+    carry += chunk_total;
+  }
+  return carry;
+}
+
+// Lanes of `act` whose key equals this lane's key, for keys below 2^key_bits:
+// one ballot per key bit, keeping the lanes that agree on every bit.  Every
+// lane of `act` must call it.
+__device__ __forceinline__ unsigned equal_keys(unsigned act, int key, int key_bits) {
+  unsigned peers = act;
+  for (int b = 0; b < key_bits; ++b) {
+    const bool one = (key >> b) & 1;
+    const unsigned ones = __ballot_sync(act, one);
+    peers &= one ? ones : ~ones;
+  }
+  return peers;
+}
+
+// One CTA per tile: per-count histogram of the tile's rows and their count sum.
+__global__ void __launch_bounds__(kTileRows)
+    tile_hist_kernel(const int32_t* __restrict__ counts, int rows, int nb_k, int tiles,
+                     int32_t* __restrict__ hist, int32_t* __restrict__ tile_sum) {
+  extern __shared__ int32_t bins_smem[];  // nb_k + 1
+  __shared__ int scan_smem[33];
+  const int bins = nb_k + 1;
+  for (int i = threadIdx.x; i < bins; i += kTileRows) bins_smem[i] = 0;
+  __syncthreads();
+  const int r = blockIdx.x * kTileRows + threadIdx.x;
+  const int c = r < rows ? counts[r] : 0;
+  if (r < rows) atomicAdd(&bins_smem[nb_k - c], 1);
+  int total;
+  block_exclusive_scan(c, scan_smem, &total);  // the tile's sum; orders the atomics
+  for (int d = threadIdx.x; d < bins; d += kTileRows)
+    hist[size_t(d) * tiles + blockIdx.x] = bins_smem[d];
+  if (threadIdx.x == 0) tile_sum[blockIdx.x] = total;
+}
+
+// One CTA: tile sums -> tile row bases (and the grand total into
+// row_offsets[rows]); histograms -> first schedule slot of every (count, tile).
+__global__ void __launch_bounds__(kTileRows, 1)
+    tile_scan_kernel(int rows, int nb_k, int tiles, int32_t* __restrict__ hist,
+                     int32_t* __restrict__ tile_sum, int32_t* __restrict__ row_offsets) {
+  __shared__ int scan_smem[33];
+  __shared__ int buf[kScanBufInts];
+  const int total = cta_exclusive_scan_inplace(tile_sum, tiles, scan_smem, buf);
+  if (threadIdx.x == 0) row_offsets[rows] = total;
+  cta_exclusive_scan_inplace(hist, (nb_k + 1) * tiles, scan_smem, buf);
+}
+
+// One CTA per tile: row_offsets of the tile's rows, then stable placement of
+// every row at its count's slot for this tile plus the number of rows of the
+// tile before it with the same count.  Within a warp that number comes from
+// equal-key lane masks; across warps (kParallelRanks) from per-warp counts per
+// key, scanned over the warps -- shared memory for 33 tables of nb_k + 1 ints;
+// otherwise the warps take turns, each advancing per-key counters in order.
+template <bool kParallelRanks>
+__global__ void __launch_bounds__(kTileRows)
+    tile_place_kernel(const int32_t* __restrict__ counts, int rows, int nb_k, int tiles,
+                      const int32_t* __restrict__ first, const int32_t* __restrict__ tile_base,
+                      int32_t* __restrict__ row_offsets, int32_t* __restrict__ schedule) {
+  extern __shared__ int32_t place_smem[];
+  __shared__ int scan_smem[33];
+  const int bins = nb_k + 1;
+  int32_t* next_slot = place_smem;          // [bins], indexed by nb_k - count
+  int32_t* warp_hist = place_smem + bins;  // [kTileWarps][bins] (kParallelRanks)
+  const int t = blockIdx.x;
+  for (int d = threadIdx.x; d < bins; d += kTileRows) next_slot[d] = first[size_t(d) * tiles + t];
+  if (kParallelRanks)
+    for (int i = threadIdx.x; i < kTileWarps * bins; i += kTileRows) warp_hist[i] = 0;
+  const int r = t * kTileRows + threadIdx.x;
+  const bool active = r < rows;
+  const int c = active ? counts[r] : 0;
+  int tile_total;
+  const int pre = block_exclusive_scan(c, scan_smem, &tile_total);  // also publishes the tables
+  if (active) row_offsets[r] = tile_base[t] + pre;
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned below = (1u << lane) - 1u;
+  const int key_bits = 32 - __clz(nb_k);  // keys d = nb_k - c lie in [0, nb_k]
+  const unsigned act = __ballot_sync(0xffffffffu, active);
+  const int d = nb_k - c;
+  if (kParallelRanks) {
+    unsigned peers = 0;
+    if (active) {
+      peers = equal_keys(act, d, key_bits);
+      if ((peers & below) == 0) warp_hist[warp * bins + d] = __popc(peers);
+    }
+    __syncthreads();
+    for (int k = threadIdx.x; k < bins; k += kTileRows) {  // exclusive scan over the warps
+      int run = 0;
+      for (int w = 0; w < kTileWarps; ++w) {
+        const int x = warp_hist[w * bins + k];
+        warp_hist[w * bins + k] = run;
+        run += x;
+      }
+    }
+    __syncthreads();
+    if (active) schedule[next_slot[d] + warp_hist[warp * bins + d] + __popc(peers & below)] = r;
+  } else {
+    for (int w = 0; w < kTileWarps; ++w) {
+      if (warp == w && active) {
+        const unsigned peers = equal_keys(act, d, key_bits);
+        const int rank = __popc(peers & below);
+        const int pos = next_slot[d] + rank;
+        schedule[pos] = r;
+        __syncwarp(act);
+        if (rank == 0) next_slot[d] = pos + __popc(peers);
+      }
+      __syncthreads();
+    }
   }
 }
 
+// One warp per row.  The row's words are loaded one per lane, then taken one
+// at a time (broadcast by shuffle): lane j owns key block 32*w + j and, if the
+// bit is set, writes it at the row's running offset plus the number of set
+// bits below it, so each store instruction writes consecutive addresses.
 __global__ void __launch_bounds__(256) write_lists_kernel(const uint32_t* __restrict__ bits,
-                                                          int64_t rows, int words,
+                                                          int rows, int words,
                                                           const int32_t* __restrict__ row_offsets,
                                                           int32_t* __restrict__ col_idx) {
   const int lane = threadIdx.x & 31;
-  const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t n_warps = (int64_t(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t r = warp; r < rows; r += n_warps) {
-    const uint32_t* row = bits + r * words;
+  const uint32_t below = (1u << lane) - 1u;
+  const int n_warps = gridDim.x * kRowWarps;
+  for (int r = blockIdx.x * kRowWarps + (threadIdx.x >> 5); r < rows; r += n_warps) {
+    const uint32_t* row = bits + size_t(r) * words;
     int out = row_offsets[r];
     for (int w0 = 0; w0 < words; w0 += 32) {
-      const int w = w0 + lane;
-      uint32_t word = w < words ? row[w] : 0u;
-      const int pc = __popc(word);
-      int incl = pc;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+      const uint32_t mine = w0 + lane < words ? row[w0 + lane] : 0u;
+      const int n = min(32, words - w0);
+      for (int k = 0; k < n; ++k) {
+        const uint32_t word = __shfl_sync(0xffffffffu, mine, k);
+        if ((word >> lane) & 1u) col_idx[out + __popc(word & below)] = (w0 + k) * 32 + lane;
+        out += __popc(word);
       }
-      int pos = out + incl - pc;
-      while (word) {  // ascending: clear the lowest set bit each step
-        col_idx[pos++] = w * 32 + (__ffs(word) - 1);
-        word &= word - 1u;
-      }
-      out += __shfl_sync(0xffffffffu, incl, 31);
     }
   }
+}
+
+int num_tiles(int64_t rows) { return int((rows + kTileRows - 1) / kTileRows); }
+
+// Workspace ints: the (count, tile) table and the tile sums.
+int64_t workspace_ints(int64_t rows, int nb_k) {
+  const int64_t tiles = num_tiles(rows);
+  return (int64_t(nb_k) + 1) * tiles + tiles;
+}
+
+// Grid of the row-parallel launches: kRowWarps warps per block, one row per
+// warp, so that every row's loads are in flight at once and blocks turn over
+// as rows finish (the kernels still stride over rows past the grid).
+int row_grid(int64_t rows) {
+  const int64_t want_blocks = (rows + kRowWarps - 1) / kRowWarps;
+  return int(want_blocks < (int64_t(1) << 30) ? want_blocks : (int64_t(1) << 30));
+}
+
+// Checks shared by every packing entry point (before any CUDA call).
+bsa_status check_pack_args(int B, int H, int nb_q, int nb_k, const void* bits,
+                           const void* counts, const void* row_offsets, const void* col_idx,
+                           const void* schedule) {
+  if (!bits || !counts || !row_offsets || !schedule) return BSA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || nb_q <= 0 || nb_k <= 0) return BSA_ERR_INVALID_ARG;
+  const int64_t rows = int64_t(B) * H * nb_q;
+  if (rows * int64_t(nb_k) >= (int64_t(1) << 31)) return BSA_ERR_OVERFLOW;
+  if (nb_k + 1 > kMaxBins) return BSA_ERR_UNSUPPORTED;
+  if (!bsa::aligned4(bits) || !bsa::aligned4(counts) || !bsa::aligned4(row_offsets) ||
+      !bsa::aligned4(schedule) || (col_idx && !bsa::aligned4(col_idx)))
+    return BSA_ERR_MISALIGNED;
+  return BSA_OK;
+}
+
+// Launches 2-5, after counts and bits of every row have been written.
+// `scratch` holds workspace_ints(rows, nb_k) ints; its contents on entry do
+// not matter (every entry is written before it is read).
+bsa_status launch_offsets_schedule_lists(const uint32_t* bits, const int32_t* counts, int rows,
+                                         int nb_k, int words, int32_t* row_offsets,
+                                         int32_t* col_idx, int32_t* schedule, int32_t* scratch,
+                                         cudaStream_t s) {
+  const int tiles = num_tiles(rows);
+  const int bins = nb_k + 1;
+  int32_t* table = scratch;                       // [bins][tiles]
+  int32_t* tile_sum = scratch + size_t(bins) * tiles;  // [tiles]
+  const size_t bins_bytes = size_t(bins) * sizeof(int32_t);
+  const size_t ranks_bytes = size_t(kTileWarps + 1) * bins_bytes;
+  const bool parallel_ranks = ranks_bytes <= kMaxDynamicSmem;
+  const size_t place_bytes = parallel_ranks ? ranks_bytes : bins_bytes;
+  if (cudaFuncSetAttribute(tile_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(bins_bytes)) != cudaSuccess)
+    return BSA_ERR_LAUNCH;
+  const cudaError_t attr =
+      parallel_ranks ? cudaFuncSetAttribute(tile_place_kernel<true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            int(place_bytes))
+                     : cudaFuncSetAttribute(tile_place_kernel<false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            int(place_bytes));
+  if (attr != cudaSuccess) return BSA_ERR_LAUNCH;
+  tile_hist_kernel<<<tiles, kTileRows, bins_bytes, s>>>(counts, rows, nb_k, tiles, table,
+                                                       tile_sum);
+  if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
+  tile_scan_kernel<<<1, kTileRows, 0, s>>>(rows, nb_k, tiles, table, tile_sum, row_offsets);
+  if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
+  if (parallel_ranks)
+    tile_place_kernel<true><<<tiles, kTileRows, place_bytes, s>>>(
+        counts, rows, nb_k, tiles, table, tile_sum, row_offsets, schedule);
+  else
+    tile_place_kernel<false><<<tiles, kTileRows, place_bytes, s>>>(
+        counts, rows, nb_k, tiles, table, tile_sum, row_offsets, schedule);
+  if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
+  if (col_idx) {
+    write_lists_kernel<<<row_grid(rows), 256, 0, s>>>(bits, rows, words, row_offsets, col_idx);
+    if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
+  }
+  return BSA_OK;
 }
 
 }  // namespace
 
 extern "C" size_t bsa_pack_mask_workspace(int B, int H, int nb_q, int nb_k) {
-  (void)B;
-  (void)H;
-  (void)nb_q;
-  if (nb_k <= 0) return 0;
-  size_t bytes = size_t(kSortWarps) * size_t(nb_k + 1) * sizeof(int32_t);
+  if (B <= 0 || H <= 0 || nb_q <= 0 || nb_k <= 0) return 0;
+  const size_t bytes =
+      size_t(workspace_ints(int64_t(B) * H * nb_q, nb_k)) * sizeof(int32_t);
   return (bytes + 255) & ~size_t(255);
 }
 
@@ -190,39 +414,54 @@ extern "C" bsa_status bsa_pack_mask(const uint8_t* dense, int B, int H, int nb_q
                                     uint32_t* bits, int32_t* counts, int32_t* row_offsets,
                                     int32_t* col_idx, int32_t* schedule, void* workspace,
                                     size_t workspace_bytes, void* stream) {
-  if (!dense || !bits || !counts || !row_offsets || !schedule) return BSA_ERR_INVALID_ARG;
-  if (B <= 0 || H <= 0 || nb_q <= 0 || nb_k <= 0) return BSA_ERR_INVALID_ARG;
-  const int64_t rows = int64_t(B) * H * nb_q;
-  if (rows * int64_t(nb_k) >= (int64_t(1) << 31)) return BSA_ERR_OVERFLOW;
-  if (!bsa::aligned4(bits) || !bsa::aligned4(counts) || !bsa::aligned4(row_offsets) ||
-      !bsa::aligned4(schedule) || (col_idx && !bsa::aligned4(col_idx)))
-    return BSA_ERR_MISALIGNED;
+  if (!dense) return BSA_ERR_INVALID_ARG;
+  const bsa_status st = check_pack_args(B, H, nb_q, nb_k, bits, counts, row_offsets, col_idx,
+                                        schedule);
+  if (st != BSA_OK) return st;
   const size_t need = bsa_pack_mask_workspace(B, H, nb_q, nb_k);
   if (!workspace || workspace_bytes < need) return BSA_ERR_WORKSPACE;
   if (!bsa::aligned16(workspace)) return BSA_ERR_MISALIGNED;
-  const int sms = bsa::num_sms();
-  if (sms <= 0) return BSA_ERR_LAUNCH;
+  if (bsa::num_sms() <= 0) return BSA_ERR_LAUNCH;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int rows = B * H * nb_q;
   const int words = (nb_k + 31) / 32;
-  const int64_t want_blocks = (rows + 7) / 8;  // 8 warps per block
-  const int grid = int(want_blocks < int64_t(sms) * 8 ? want_blocks : int64_t(sms) * 8);
-  pack_rows_kernel<<<grid, 256, 0, s>>>(dense, rows, nb_k, words, bits, counts);
+  pack_rows_kernel<<<row_grid(rows), 256, 0, s>>>(dense, rows, nb_k, words, bits, counts);
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
-  scan_sort_kernel<<<1, kSortThreads, 0, s>>>(counts, int(rows), nb_k, row_offsets, schedule,
-                                               static_cast<int32_t*>(workspace));
+  return launch_offsets_schedule_lists(bits, counts, rows, nb_k, words, row_offsets, col_idx,
+                                       schedule, static_cast<int32_t*>(workspace), s);
+}
+
+extern "C" bsa_status bsa_pack_mask_from_threshold(const float* thr, const float* p, int B,
+                                                   int H, int nb_q, int nb_k, uint32_t* bits,
+                                                   int32_t* counts, int32_t* row_offsets,
+                                                   int32_t* col_idx, int32_t* schedule,
+                                                   void* workspace, size_t workspace_bytes,
+                                                   void* stream) {
+  if (!thr || !p) return BSA_ERR_INVALID_ARG;
+  const bsa_status st = check_pack_args(B, H, nb_q, nb_k, bits, counts, row_offsets, col_idx,
+                                        schedule);
+  if (st != BSA_OK) return st;
+  if (!bsa::aligned4(thr) || !bsa::aligned4(p)) return BSA_ERR_MISALIGNED;
+  const size_t need = bsa_pack_mask_workspace(B, H, nb_q, nb_k);
+  if (!workspace || workspace_bytes < need) return BSA_ERR_WORKSPACE;
+  if (!bsa::aligned16(workspace)) return BSA_ERR_MISALIGNED;
+  if (bsa::num_sms() <= 0) return BSA_ERR_LAUNCH;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int rows = B * H * nb_q;
+  const int words = (nb_k + 31) / 32;
+  pack_threshold_rows_kernel<<<row_grid(rows), 256, 0, s>>>(thr, p, nb_q, H * nb_q, rows, nb_k,
+                                                            words, bits, counts);
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
-  if (col_idx) {
-    write_lists_kernel<<<grid, 256, 0, s>>>(bits, rows, words, row_offsets, col_idx);
-    if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
-  }
-  return BSA_OK;
+  return launch_offsets_schedule_lists(bits, counts, rows, nb_k, words, row_offsets, col_idx,
+                                       schedule, static_cast<int32_t*>(workspace), s);
 }
 
 // ---------------------------------------------------------------------------
-// bsa_pack_mask_noalloc: the same three kernels as bsa_pack_mask, with the
-// sort's scratch histogram in a fixed device array that this library owns,
-// for callers that cannot allocate device memory.
+// bsa_pack_mask_noalloc: the same launches as bsa_pack_mask, with the sort's
+// scratch in a fixed device array that this library owns, for callers that
+// cannot allocate device memory.
 //
 // The array below lives in every GPU's memory from the moment the library is
 // loaded on it until the process exits (512 KiB).  Host code cannot use the
@@ -231,8 +470,7 @@ extern "C" bsa_status bsa_pack_mask(const uint8_t* dense, int B, int H, int nb_q
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr int kNoallocMaxNbK = 4095;  // key blocks per row the fixed scratch can sort
-constexpr int kNoallocScratchInts = kSortWarps * (kNoallocMaxNbK + 1);
+constexpr int kNoallocScratchInts = 131072;  // 512 KiB
 constexpr int kNoallocMaxDevices = 64;
 
 static __device__ __align__(256) int32_t g_pack_scratch[kNoallocScratchInts];
@@ -260,33 +498,23 @@ extern "C" bsa_status bsa_pack_mask_noalloc(const uint8_t* dense, int B, int H, 
                                             int nb_k, uint32_t* bits, int32_t* counts,
                                             int32_t* row_offsets, int32_t* col_idx,
                                             int32_t* schedule, void* stream) {
-  if (!dense || !bits || !counts || !row_offsets || !schedule) return BSA_ERR_INVALID_ARG;
-  if (B <= 0 || H <= 0 || nb_q <= 0 || nb_k <= 0) return BSA_ERR_INVALID_ARG;
-  if (nb_k > kNoallocMaxNbK) return BSA_ERR_WORKSPACE;  // the fixed scratch is too small
-  const int64_t rows = int64_t(B) * H * nb_q;
-  if (rows * int64_t(nb_k) >= (int64_t(1) << 31)) return BSA_ERR_OVERFLOW;
-  if (!bsa::aligned4(bits) || !bsa::aligned4(counts) || !bsa::aligned4(row_offsets) ||
-      !bsa::aligned4(schedule) || (col_idx && !bsa::aligned4(col_idx)))
-    return BSA_ERR_MISALIGNED;
+  if (!dense) return BSA_ERR_INVALID_ARG;
+  const bsa_status st = check_pack_args(B, H, nb_q, nb_k, bits, counts, row_offsets, col_idx,
+                                        schedule);
+  if (st != BSA_OK) return st;
+  // the fixed scratch must hold the (count, tile) table and the tile sums
+  if (workspace_ints(int64_t(B) * H * nb_q, nb_k) > kNoallocScratchInts) return BSA_ERR_WORKSPACE;
   int32_t* scratch = noalloc_scratch_for_current_device();
   if (!scratch) return BSA_ERR_LAUNCH;
-  const int sms = bsa::num_sms();
-  if (sms <= 0) return BSA_ERR_LAUNCH;
+  if (bsa::num_sms() <= 0) return BSA_ERR_LAUNCH;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int rows = B * H * nb_q;
   const int words = (nb_k + 31) / 32;
-  const int64_t want_blocks = (rows + 7) / 8;  // 8 warps per block
-  const int grid = int(want_blocks < int64_t(sms) * 8 ? want_blocks : int64_t(sms) * 8);
-  pack_rows_kernel<<<grid, 256, 0, s>>>(dense, rows, nb_k, words, bits, counts);
+  pack_rows_kernel<<<row_grid(rows), 256, 0, s>>>(dense, rows, nb_k, words, bits, counts);
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
-  // scan_sort_kernel zeroes the histogram part of the scratch it uses before
-  // counting, so whatever an earlier call left there does not matter
-  scan_sort_kernel<<<1, kSortThreads, 0, s>>>(counts, int(rows), nb_k, row_offsets, schedule,
-                                               scratch);
-  if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
-  if (col_idx) {
-    write_lists_kernel<<<grid, 256, 0, s>>>(bits, rows, words, row_offsets, col_idx);
-    if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
-  }
-  return BSA_OK;
+  // every scratch entry the sort reads is written earlier in the same call, so
+  // whatever an earlier call left there does not matter
+  return launch_offsets_schedule_lists(bits, counts, rows, nb_k, words, row_offsets, col_idx,
+                                       schedule, scratch, s);
 }

@@ -261,6 +261,38 @@ def gen_mask(w: Workload, q: torch.Tensor | None = None, k: torch.Tensor | None 
     raise ValueError(f"unknown mask kind {w.mask_kind}")
 
 
+THRESHOLD_LEVELS = 20  # candidate densities 0.05, 0.10, ..., 1.00
+
+
+def gen_threshold(w: Workload, seed: int | None = None):
+    """Synthetic per-head threshold map and per-head density thresholds.
+
+    Stands in for the offline Threshold Map of "ScalingAttention" Sec. 4.1.2
+    (Eq. 2; built there from calibration prompts on trained weights, which are
+    not available here) and for FAST's per-head choice of p (Algorithm 1).
+    Recipe: thresholds live on the candidate grid k/20; head h draws
+    gamma_h ~ U[0.5, 2] and block (u, v) gets ceil(20 * min(1, U^gamma_h +
+    0.03 * |slab(u) - slab(v)|)) / 20 with U ~ U[0, 1), so nearby slabs become
+    active at lower thresholds; diagonal blocks get the lowest level, 0.05.
+    p_h is drawn from the levels 0.20 .. 0.60.
+
+    Returns (thr float32 [H, nb, nb], p float32 [H])."""
+    seed = (w.seed if seed is None else seed) + 2000
+    rng = np.random.default_rng(seed)
+    slab, _ = block_coords(w.nb, w.n_slabs)
+    dslab = np.abs(slab[:, None] - slab[None, :]).astype(np.float64)
+    levels = THRESHOLD_LEVELS
+    thr = np.empty((w.H, w.nb, w.nb), dtype=np.float32)
+    for h in range(w.H):
+        gamma = rng.uniform(0.5, 2.0)
+        score = np.minimum(1.0, rng.random((w.nb, w.nb)) ** gamma + 0.03 * dslab)
+        k = np.clip(np.ceil(score * levels), 1, levels)
+        np.fill_diagonal(k, 1)
+        thr[h] = (k / levels).astype(np.float32)
+    p = (rng.integers(4, 13, size=w.H) / levels).astype(np.float32)
+    return thr, p
+
+
 def kept_tiles(mask: np.ndarray) -> int:
     return int(np.count_nonzero(mask))
 

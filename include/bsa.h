@@ -24,8 +24,9 @@
  *     traps.  A launch failure returns BSA_ERR_LAUNCH.
  *   - bf16 tensors are raw IEEE bfloat16 (2 bytes), row-major, with the shape
  *     given beside each argument; the innermost index is contiguous.
- *   - Every pointer passed to a data argument must be 16-byte aligned, else
- *     BSA_ERR_MISALIGNED.
+ *   - A data pointer must be 16-byte aligned unless the call's description
+ *     below asks for less (4-byte for the mask-packing and threshold-map
+ *     calls), else BSA_ERR_MISALIGNED.
  */
 #ifndef BSA_H_
 #define BSA_H_
@@ -87,8 +88,8 @@ const char* bsa_status_string(bsa_status status);
  *
  * Alignment: dense needs no alignment; every other pointer must be 4-byte
  * aligned (16-byte for workspace).  Errors: BSA_ERR_INVALID_ARG (null output,
- * a size <= 0), BSA_ERR_OVERFLOW (B*H*nb_q*nb_k >= 2^31),
- * BSA_ERR_WORKSPACE, BSA_ERR_LAUNCH.
+ * a size <= 0), BSA_ERR_OVERFLOW (B*H*nb_q*nb_k >= 2^31), BSA_ERR_UNSUPPORTED
+ * (nb_k > 49151), BSA_ERR_WORKSPACE, BSA_ERR_LAUNCH.
  * ------------------------------------------------------------------------- */
 size_t bsa_pack_mask_workspace(int B, int H, int nb_q, int nb_k);
 bsa_status bsa_pack_mask(const uint8_t* dense, int B, int H, int nb_q, int nb_k, uint32_t* bits,
@@ -108,8 +109,10 @@ bsa_status bsa_pack_mask(const uint8_t* dense, int B, int H, int nb_q, int nb_k,
  * scratch is a fixed 512 KiB array inside the library, present on every GPU
  * that loads it until the process exits.
  *
- * Limit: nb_k <= 4095; larger nb_k returns BSA_ERR_WORKSPACE (the built-in
- * scratch is too small; use bsa_pack_mask).  The first call on each device
+ * Limit: the built-in scratch holds 131072 ints and the call needs
+ * (nb_k + 2) * ceil(B*H*nb_q / 1024) of them (e.g. every workload with up to
+ * 40 heads of 1024 query blocks of 1024 key blocks, B = 1, fits); a larger
+ * call returns BSA_ERR_WORKSPACE (use bsa_pack_mask).  The first call on each device
  * looks up the array's device address (cudaGetSymbolAddress) with that device
  * current, so make that first call before any stream capture.  All calls share
  * the one array: calls whose kernels overlap on a GPU (for example on two
@@ -120,6 +123,64 @@ bsa_status bsa_pack_mask(const uint8_t* dense, int B, int H, int nb_q, int nb_k,
 bsa_status bsa_pack_mask_noalloc(const uint8_t* dense, int B, int H, int nb_q, int nb_k,
                                  uint32_t* bits, int32_t* counts, int32_t* row_offsets,
                                  int32_t* col_idx, int32_t* schedule, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * bsa_pack_mask_from_threshold -- threshold map + per-head density threshold
+ * -> CRM rows + lists + schedule, with no dense mask in between.
+ *
+ * Follows Sec. 4.1.2 (Eq. 2): the Threshold Map T records, per block (u, v),
+ * the smallest sparsity threshold at which the block is active, and a mask for
+ * a target threshold p is M_p = 1(T <= p).  Algorithm 1 (FAST, mask
+ * instantiation) picks one p per layer, timestep and head, so p holds one
+ * value per head and the map is shared by all batch items.  The result is
+ * exactly bsa_pack_mask applied to the dense mask
+ *     dense[b, h, u, v] = (thr[h, u, v] <= p[h]) ? 1 : 0
+ * (fp32 comparison; a NaN threshold or a NaN p keeps nothing).
+ *
+ *   thr   [H, nb_q, nb_k] fp32 device array, 4-byte aligned.
+ *   p     [H] fp32 device array, 4-byte aligned.
+ *   bits, counts, row_offsets, col_idx, schedule, workspace: as for
+ *         bsa_pack_mask (same shapes, same workspace size from
+ *         bsa_pack_mask_workspace(B, H, nb_q, nb_k)).
+ *
+ * Errors: BSA_ERR_INVALID_ARG (null pointer, a size <= 0), BSA_ERR_MISALIGNED,
+ * BSA_ERR_OVERFLOW (B*H*nb_q*nb_k >= 2^31), BSA_ERR_WORKSPACE, BSA_ERR_LAUNCH.
+ * ------------------------------------------------------------------------- */
+bsa_status bsa_pack_mask_from_threshold(const float* thr, const float* p, int B, int H, int nb_q,
+                                        int nb_k, uint32_t* bits, int32_t* counts,
+                                        int32_t* row_offsets, int32_t* col_idx,
+                                        int32_t* schedule, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * bsa_threshold_resize -- resize a threshold map to another block grid
+ * (Sec. 4.3.1, Eq. 7: the map of a base resolution is resized by conservative
+ * bilinear interpolation with a ceiling rule, so that any overlap with an
+ * active region is preserved; the topology is built once and reused at every
+ * resolution).
+ *
+ * Target block (u, v) samples the source map at (u * sq / tq, v * sk / tk).
+ * Along each axis the source blocks with a nonzero bilinear weight are
+ * floor(u * sq / tq) and, when u * sq is not a multiple of tq, the next block
+ * (clamped to sq - 1); likewise for v.  The ceiling of the bilinearly
+ * resampled indicator 1(T <= p) is 1 exactly when one of those blocks is
+ * active, for every p; so the target threshold is their minimum:
+ *     dst[h, u, v] = min over those (a, c) of src[h, a, c]
+ * NaN entries are skipped; if all are NaN the result is NaN; when +0 and -0
+ * tie, the sign of the zero returned is unspecified (no mask can tell them
+ * apart).  Exact (no arithmetic on the thresholds), so pack(resize(T), p)
+ * equals the ceiling rule applied to pack(T, p) at every p.
+ *
+ *   src [H, sq, sk] fp32 device array, dst [H, tq, tk] fp32 device array;
+ *   both 4-byte aligned, not overlapping.  Sizes 1 .. 65535 per axis (up- or
+ *   downscale).
+ *
+ * Errors: BSA_ERR_INVALID_ARG (null pointer, a size <= 0), BSA_ERR_UNSUPPORTED
+ * (a size above 65535), BSA_ERR_MISALIGNED, BSA_ERR_OVERFLOW (H*tq >= 2^31),
+ * BSA_ERR_LAUNCH.
+ * ------------------------------------------------------------------------- */
+bsa_status bsa_threshold_resize(const float* src, int H, int sq, int sk, float* dst, int tq,
+                                int tk, void* stream);
 
 /* ---------------------------------------------------------------------------
  * bsa_tile_permute / bsa_tile_unpermute -- 3-D tile gather (Sec. 5.4-5.5,

@@ -59,6 +59,37 @@ def test_pack_mask_rejects_bad_args(lib):
     assert lib.bsa_pack_mask(fake, 1, 1, 4, 4, fake, fake, fake, fake, fake, fake, 1, None) == 7
 
 
+def test_pack_from_threshold_rejects_bad_args(lib):
+    P = ctypes.c_void_p
+    f = P(0x1000)
+    fn = lib.bsa_pack_mask_from_threshold
+    # null threshold map, null p
+    assert fn(None, f, 1, 1, 4, 4, f, f, f, f, f, f, 4096, None) == 1
+    assert fn(f, None, 1, 1, 4, 4, f, f, f, f, f, f, 4096, None) == 1
+    # non-positive batch
+    assert fn(f, f, 0, 1, 4, 4, f, f, f, f, f, f, 4096, None) == 1
+    # int32 overflow of B*H*nb_q*nb_k
+    assert fn(f, f, 64, 64, 1024, 1024, f, f, f, f, f, f, 1 << 30, None) == 4
+    # misaligned map or p
+    assert fn(P(0x1002), f, 1, 1, 4, 4, f, f, f, f, f, f, 4096, None) == 3
+    assert fn(f, P(0x1001), 1, 1, 4, 4, f, f, f, f, f, f, 4096, None) == 3
+    # workspace too small
+    assert fn(f, f, 1, 1, 4, 4, f, f, f, f, f, f, 1, None) == 7
+
+
+def test_threshold_resize_rejects_bad_args(lib):
+    P = ctypes.c_void_p
+    a, b = P(0x1000), P(0x2000)
+    fn = lib.bsa_threshold_resize
+    assert fn(None, 1, 4, 4, b, 8, 8, None) == 1
+    assert fn(a, 1, 4, 4, None, 8, 8, None) == 1
+    assert fn(a, 1, 0, 4, b, 8, 8, None) == 1
+    assert fn(a, 1, 4, 4, b, 8, -1, None) == 1
+    assert fn(P(0x1001), 1, 4, 4, b, 8, 8, None) == 3
+    assert fn(a, 1, 4, 4, b, 65536, 8, None) == 2  # more blocks per axis than supported
+    assert fn(a, 1 << 20, 4, 4, b, 4096, 8, None) == 4  # H * tq >= 2^31
+
+
 def test_permute_rejects_bad_args(lib):
     P = ctypes.c_void_p
     a, b = P(0x1000), P(0x2000)

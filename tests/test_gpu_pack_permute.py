@@ -36,7 +36,8 @@ def test_pack_mask_workloads(cuda_ok, name):
 
 @pytest.mark.parametrize("shape,density", [((1, 1, 1, 1), 1.0), ((1, 3, 5, 33), 0.3),
                                            ((2, 3, 64, 64), 0.0), ((1, 2, 100, 65), 0.9),
-                                           ((1, 4, 990, 990), 0.12), ((3, 1, 7, 1100), 0.5)])
+                                           ((1, 4, 990, 990), 0.12), ((3, 1, 7, 1100), 0.5),
+                                           ((1, 2, 40, 2000), 0.4)])
 def test_pack_mask_edge_shapes(cuda_ok, shape, density):
     rng = np.random.default_rng(sum(shape))
     dense = (rng.random(shape) < density).astype(np.uint8)

@@ -68,10 +68,12 @@ def test_noalloc_pack_matches_pack_mask_twice_in_a_row(cuda_ok):
         assert total == int(np.count_nonzero(m))
 
 
-def test_noalloc_rejects_rows_longer_than_its_scratch(cuda_ok):
+def test_noalloc_rejects_masks_larger_than_its_scratch(cuda_ok):
+    # 262144 rows -> 256 tiles of 1024 rows, times (600 + 2) ints > 131072:
+    # rejected on the host, before any launch (the pointers are never used)
     from block_sparse_attention_forward_b200 import _ffi
     lib = _ffi.load()
     P = ctypes.c_void_p
     fake = P(0x1000)
-    assert lib.bsa_pack_mask_noalloc(fake, 1, 1, 1, 4096, fake, fake, fake, fake, fake,
+    assert lib.bsa_pack_mask_noalloc(fake, 1, 64, 4096, 600, fake, fake, fake, fake, fake,
                                      None) == 7  # BSA_ERR_WORKSPACE
