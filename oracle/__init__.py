@@ -23,6 +23,11 @@ Intrinsic Sparse Attention Topology for Video Diffusion Transformers"):
                             threshold per head (Algorithm 1, FAST).
 - ``threshold_resize``   -- Sec. 4.3.1, Eq. 7 (conservative bilinear resize of
                             the threshold map with the ceiling rule).
+- ``hilbert_key``, ``hilbert_order``
+                         -- DFSAttn's Hilbert-curve token reordering, as a 3-D
+                            Hilbert curve over the enclosing power-of-two cube
+                            (Skilling's transpose method), grid points in curve
+                            order.
 """
 from __future__ import annotations
 
@@ -75,6 +80,10 @@ def _load():
                                              P, I64, I, P, P]
             lib.oracle_threshold_mask.argtypes = [P, P, I, I, I, I, P]
             lib.oracle_threshold_resize.argtypes = [P, I, I, I, P, I, I]
+            lib.oracle_hilbert_key.argtypes = [I, I, I, I]
+            lib.oracle_hilbert_key.restype = ctypes.c_uint64
+            lib.oracle_hilbert_order.argtypes = [I, I, I, P]
+            lib.oracle_hilbert_order.restype = I
             _lib = lib
     return _lib
 
@@ -202,3 +211,16 @@ def threshold_resize(src: np.ndarray, tq: int, tk: int) -> np.ndarray:
     dst = np.empty((H, tq, tk), dtype=np.float32)
     _load().oracle_threshold_resize(_ptr(src), H, sq, sk, _ptr(dst), int(tq), int(tk))
     return dst
+
+
+def hilbert_key(t: int, y: int, x: int, bits: int) -> int:
+    """Index of (t, y, x) on the 3-D Hilbert curve over the cube of side 2**bits."""
+    return int(_load().oracle_hilbert_key(int(t), int(y), int(x), int(bits)))
+
+
+def hilbert_order(T: int, Hs: int, Ws: int) -> np.ndarray:
+    """perm[p] = frame-major index of the token at position p of the Hilbert order."""
+    perm = np.zeros(T * Hs * Ws, dtype=np.int64)
+    if _load().oracle_hilbert_order(T, Hs, Ws, _ptr(perm)) < 0:
+        raise MemoryError("oracle_hilbert_order")
+    return perm

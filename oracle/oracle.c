@@ -351,3 +351,86 @@ void oracle_threshold_resize(const float* src, int H, int sq, int sk, float* dst
       }
     }
 }
+
+/* ------------------------------------------------------------------ */
+/* Hilbert-curve token order (DFSAttn: Hilbert curve-based token       */
+/* reordering; used with block-sparse attention as in ScalingAttention */
+/* Sec. 5.4-5.5, token permutation into hardware-friendly blocks).     */
+/*                                                                     */
+/* The curve is the 3-D Hilbert curve over the cube of side 2^bits     */
+/* that encloses the T x Hs x Ws grid, axes (t, y, x); grid points are */
+/* taken in curve order and points outside the grid are skipped.  The  */
+/* index of a point follows J. Skilling, "Programming the Hilbert      */
+/* curve" (AIP Conf. Proc. 707, 2004): the axes are turned into the    */
+/* "transpose" of the index by undoing, from the top level down, the   */
+/* inversions and exchanges the inverse map would make, then Gray      */
+/* coding across the axes; the index reads the transpose bit by bit,   */
+/* top level first, axis t first.                                      */
+/* ------------------------------------------------------------------ */
+static uint64_t hilbert_key(const uint32_t axes_in[3], int bits) {
+  uint32_t a[3] = {axes_in[0], axes_in[1], axes_in[2]};
+  for (int level = bits - 1; level >= 1; --level) {
+    const uint32_t bit = 1u << level;
+    const uint32_t below = bit - 1u;
+    for (int i = 0; i < 3; ++i) {
+      if ((a[i] & bit) != 0) {
+        a[0] ^= below; /* inversion of the low bits of axis 0 */
+      } else {
+        const uint32_t diff = (a[0] ^ a[i]) & below; /* exchange low bits of 0 and i */
+        a[0] ^= diff;
+        a[i] ^= diff;
+      }
+    }
+  }
+  for (int i = 1; i < 3; ++i) a[i] ^= a[i - 1]; /* Gray code across the axes */
+  uint32_t flip = 0;
+  for (int level = bits - 1; level >= 1; --level)
+    if ((a[2] & (1u << level)) != 0) flip ^= (1u << level) - 1u;
+  for (int i = 0; i < 3; ++i) a[i] ^= flip;
+  uint64_t key = 0;
+  for (int level = bits - 1; level >= 0; --level)
+    for (int i = 0; i < 3; ++i) key = (key << 1) | (uint64_t)((a[i] >> level) & 1u);
+  return key;
+}
+
+typedef struct {
+  uint64_t key;
+  int64_t frame;
+} keyed_token;
+
+static int cmp_keyed(const void* pa, const void* pb) {
+  const keyed_token* a = (const keyed_token*)pa;
+  const keyed_token* b = (const keyed_token*)pb;
+  if (a->key < b->key) return -1;
+  if (a->key > b->key) return 1;
+  return 0;
+}
+
+/* Hilbert key of a point on the cube of side 2^bits (exposed for the pins). */
+uint64_t oracle_hilbert_key(int t, int y, int x, int bits) {
+  const uint32_t axes[3] = {(uint32_t)t, (uint32_t)y, (uint32_t)x};
+  return hilbert_key(axes, bits);
+}
+
+/* perm[p] = frame-major index of the token at position p of the Hilbert order.
+ * Returns the number of bits per axis of the enclosing cube. */
+int oracle_hilbert_order(int T, int Hs, int Ws, int64_t* perm) {
+  int side = T > Hs ? T : Hs;
+  if (Ws > side) side = Ws;
+  int bits = 1;
+  while ((1 << bits) < side) ++bits;
+  const int64_t n = (int64_t)T * Hs * Ws;
+  keyed_token* tok = (keyed_token*)malloc((size_t)n * sizeof(keyed_token));
+  if (!tok) return -1;
+  for (int t = 0; t < T; ++t)
+    for (int y = 0; y < Hs; ++y)
+      for (int x = 0; x < Ws; ++x) {
+        const int64_t f = ((int64_t)t * Hs + y) * Ws + x;
+        tok[f].key = oracle_hilbert_key(t, y, x, bits);
+        tok[f].frame = f;
+      }
+  qsort(tok, (size_t)n, sizeof(keyed_token), cmp_keyed);
+  for (int64_t i = 0; i < n; ++i) perm[i] = tok[i].frame;
+  free(tok);
+  return bits;
+}
