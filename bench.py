@@ -16,9 +16,10 @@ shape (different seed): the path shards by (batch, head) with no exchange, so
 there is no collective on the data path (weak scaling); the step time is the
 max over ranks.
 
-After the timed steps, `next_rows` reports the threshold-map steps measured
-on their own (L2 flushed before each call): bsa_pack_mask_from_threshold at the
-workload's block grid and bsa_threshold_resize of a 480p-grid map to it.
+After the timed steps, `next_rows` reports further steps measured on their own
+(L2 flushed before each call): bsa_pack_mask_from_threshold at the workload's
+block grid, bsa_threshold_resize of a 480p-grid map to it, and bsa_gather_rows
+applying the Hilbert-curve order and head-aware tile orders to one tensor.
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of query blocks of the same workload (rank 0 only).
@@ -289,6 +290,39 @@ def measure_threshold_rows(w, dev, stream, hbm_gbs: float):
     }
 
 
+HEAD_TILES = [(1, 8, 16), (2, 8, 8), (4, 4, 8), (1, 16, 8)]  # synthetic head-aware shapes
+
+
+def measure_order_rows(w, dev, stream, hbm_gbs: float):
+    """Other token orders, applied by bsa_gather_rows to one [B, H, N, d] bf16
+    tensor of the workload: the Hilbert-curve order (one table) and head-aware
+    tiles (head h uses HEAD_TILES[h % 4], one table per head).  HBM-bound;
+    algorithmic bytes = N rows read + n_pad rows written per head (the tables,
+    4 bytes per position, are not counted)."""
+    import block_sparse_attention_forward_b200 as bsa
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    g = torch.Generator().manual_seed(w.seed + 3000)
+    x = torch.randn((w.B, w.H, w.n, w.d), generator=g).to(torch.bfloat16).to(dev)
+    out = torch.empty((w.B, w.H, w.n_pad, w.d), dtype=torch.bfloat16, device=dev)
+    hil, _ = bsa.order_tables(bsa.hilbert_order(w.T, w.Hs, w.Ws), w.n_pad)
+    hil = hil.to(dev)
+    per_head = torch.stack([
+        bsa.order_tables(bsa.tile_order(w.T, w.Hs, w.Ws, *HEAD_TILES[h % 4]), w.n_pad)[0]
+        for h in range(w.H)]).to(dev)
+    row_bytes = w.d * 2
+    nbytes = w.B * w.H * (w.n + w.n_pad) * row_bytes
+    res = {}
+    for name, table in (("permute_hilbert", hil), ("permute_head_aware", per_head)):
+        us = time_device_us(lambda: bsa.gather_rows(x, table, out=out), stream, flush)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        res[name] = {"us": us, "bytes": nbytes, "achieved_gbs": gbs, "frac_hbm": gbs / hbm_gbs,
+                     "bound": "hbm", "launches": 1,
+                     "l2": "flushed before each call (the tensor is also larger than L2)"}
+    res["permute_head_aware"]["tiles"] = [list(t) for t in HEAD_TILES]
+    del flush, x, out
+    return res
+
+
 def workload_config(w, mask):
     kept = I.kept_tiles(mask)
     total = w.B * w.H * w.nb * w.nb
@@ -332,6 +366,8 @@ def main():
         peaks, _ = load_peaks()
         rows = measure_threshold_rows(w, dev, torch.cuda.current_stream(dev),
                                       float(peaks["hbm_gbs"]))
+        rows.update(measure_order_rows(w, dev, torch.cuda.current_stream(dev),
+                                       float(peaks["hbm_gbs"])))
         if rank == 0:
             print(json.dumps({"workload": w.name, "next_rows": rows}), flush=True)
         if world > 1:
@@ -455,6 +491,7 @@ def main():
     next_rows = None
     if not args.no_next:
         next_rows = measure_threshold_rows(w, dev, stream, float(peaks["hbm_gbs"]))
+        next_rows.update(measure_order_rows(w, dev, stream, float(peaks["hbm_gbs"])))
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",

@@ -9,6 +9,12 @@ devices and contiguity, then passes raw pointers to the library.
     qp = tile_permute(q, grid, tile, n_pad)        # frame-major -> 3-D tiles
     out_p, lse = forward(qp, kp, vp, mask, n_valid, block)
     out = tile_unpermute(out_p, grid, tile)        # back to frame-major
+
+Other token orders (Hilbert curve, one tile shape per head) are host-built
+tables applied on the GPU by one gather:
+
+    fwd, inv = order_tables(hilbert_order(T, Hs, Ws), n_pad)
+    qp = gather_rows(q, fwd.cuda(), n_pad)         # and gather_rows(out_p, inv.cuda(), N)
 """
 from __future__ import annotations
 
@@ -21,8 +27,8 @@ from . import _ffi
 from ._ffi import BsaError, BsaMask
 
 __all__ = ["BsaError", "PackedMask", "pack_mask", "pack_mask_from_threshold",
-           "threshold_resize", "tile_permute", "tile_unpermute", "forward", "device_error",
-           "version"]
+           "threshold_resize", "tile_permute", "tile_unpermute", "hilbert_order", "tile_order",
+           "order_tables", "gather_rows", "forward", "device_error", "version"]
 
 
 def _stream(device: torch.device) -> ctypes.c_void_p:
@@ -175,6 +181,63 @@ def tile_unpermute(y: torch.Tensor, grid, tile, out: torch.Tensor | None = None)
     st = _ffi.load().bsa_tile_unpermute(y.data_ptr(), out.data_ptr(), B, H, T, Hs, Ws, d, tt, th,
                                         tw, n_pad, _stream(y.device))
     _ffi.check(st, "bsa_tile_unpermute")
+    return out
+
+
+def _host_i32(n: int) -> torch.Tensor:
+    return torch.empty(n, dtype=torch.int32)
+
+
+def hilbert_order(T: int, Hs: int, Ws: int) -> torch.Tensor:
+    """Host int32 [T*Hs*Ws]: frame-major token index at each position of the 3-D
+    Hilbert-curve order (bsa_hilbert_order)."""
+    order = _host_i32(T * Hs * Ws)
+    _ffi.check(_ffi.load().bsa_hilbert_order(T, Hs, Ws, order.data_ptr()), "bsa_hilbert_order")
+    return order
+
+
+def tile_order(T: int, Hs: int, Ws: int, tt: int, th: int, tw: int) -> torch.Tensor:
+    """Host int32 [T*Hs*Ws]: the tile order of bsa_tile_permute as a table (bsa_tile_order)."""
+    order = _host_i32(T * Hs * Ws)
+    _ffi.check(_ffi.load().bsa_tile_order(T, Hs, Ws, tt, th, tw, order.data_ptr()),
+               "bsa_tile_order")
+    return order
+
+
+def order_tables(order: torch.Tensor, n_pad: int):
+    """Host order int32 [n] -> host gather tables (fwd int32 [n_pad], inv int32 [n])
+    (bsa_order_tables).  Stack per-head tables into [H, n_pad] for gather_rows."""
+    order = order.to(torch.int32).contiguous()
+    if order.is_cuda or order.dim() != 1:
+        raise ValueError("order must be a 1-D host tensor")
+    n = order.numel()
+    fwd, inv = _host_i32(n_pad), _host_i32(n)
+    _ffi.check(_ffi.load().bsa_order_tables(order.data_ptr(), n, int(n_pad), fwd.data_ptr(),
+                                            inv.data_ptr()), "bsa_order_tables")
+    return fwd, inv
+
+
+def gather_rows(x: torch.Tensor, src: torch.Tensor, n_out: int | None = None,
+                out: torch.Tensor | None = None) -> torch.Tensor:
+    """[B, H, n_in, d] bf16 -> [B, H, n_out, d]: row i of each head is row src[i]
+    (src [n_out] shared, or [H, n_out] per head, int32 on the GPU); entries
+    outside [0, n_in) give zero rows (bsa_gather_rows)."""
+    _require_cuda(x, "x", torch.bfloat16)
+    _require_cuda(src, "src", torch.int32)
+    B, H, n_in, d = x.shape
+    per_head = 1 if src.dim() == 2 else 0
+    if per_head and src.shape[0] != H:
+        raise ValueError("a per-head table must be [H, n_out]")
+    n_tab = src.shape[-1]
+    n_out = n_tab if n_out is None else int(n_out)
+    if n_out != n_tab:
+        raise ValueError("n_out must match the table length")
+    if out is None:
+        out = torch.empty((B, H, n_out, d), dtype=x.dtype, device=x.device)
+    _require_cuda(out, "out", torch.bfloat16)
+    st = _ffi.load().bsa_gather_rows(x.data_ptr(), out.data_ptr(), B, H, n_in, n_out, d,
+                                     src.data_ptr(), per_head, _stream(x.device))
+    _ffi.check(st, "bsa_gather_rows")
     return out
 
 

@@ -31,6 +31,10 @@ EXPORTED = (
     "bsa_pack_mask_noalloc",
     "bsa_pack_mask_from_threshold",
     "bsa_threshold_resize",
+    "bsa_hilbert_order",
+    "bsa_tile_order",
+    "bsa_order_tables",
+    "bsa_gather_rows",
     "bsa_tile_permute",
     "bsa_tile_unpermute",
     "bsa_forward",
@@ -86,6 +90,14 @@ def load() -> ctypes.CDLL:
     lib.bsa_pack_mask_from_threshold.restype = I
     lib.bsa_threshold_resize.argtypes = [P, I, I, I, P, I, I, P]
     lib.bsa_threshold_resize.restype = I
+    lib.bsa_hilbert_order.argtypes = [I, I, I, P]
+    lib.bsa_hilbert_order.restype = I
+    lib.bsa_tile_order.argtypes = [I, I, I, I, I, I, P]
+    lib.bsa_tile_order.restype = I
+    lib.bsa_order_tables.argtypes = [P, I, I, P, P]
+    lib.bsa_order_tables.restype = I
+    lib.bsa_gather_rows.argtypes = [P, P, I, I, I, I, I, P, I, P]
+    lib.bsa_gather_rows.restype = I
     for name in ("bsa_tile_permute", "bsa_tile_unpermute"):
         fn = getattr(lib, name)
         fn.argtypes = [P, P, I, I, I, I, I, I, I, I, I, I, P]

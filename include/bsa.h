@@ -208,6 +208,54 @@ bsa_status bsa_tile_unpermute(const void* in, void* out, int B, int H, int T, in
                               int d, int tt, int th, int tw, int n_pad, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Token orders as tables, and the gather that applies them.
+ *
+ * Token permutation eases the 128 x 128 granularity bottleneck by clustering
+ * related tokens into the same block (Sec. 5.4-5.5).  Besides the 3-D tile
+ * order above, the pages name DFSAttn's Hilbert curve-based token reordering
+ * and Veda's head-aware tiling (heads with differently shaped tiles).  An
+ * order is fixed per grid shape, so it is built once on the HOST as a table
+ * (these three calls take and fill host arrays, run on the calling thread and
+ * touch no GPU); each step then applies it on the GPU with bsa_gather_rows.
+ * An order lists, for each position p of the new order, the frame-major index
+ * (t*Hs + y)*Ws + x of the token placed there.
+ *
+ * bsa_hilbert_order: order[N] (host) of the 3-D Hilbert curve over the cube of
+ *   side 2^bits >= max(T, Hs, Ws), axes (t, y, x), points outside the grid
+ *   skipped; the Hilbert index follows J. Skilling, "Programming the Hilbert
+ *   curve" (2004).  Errors: BSA_ERR_INVALID_ARG (null, a size <= 0,
+ *   N >= 2^31), BSA_ERR_UNSUPPORTED (a side above 2^21).
+ * bsa_tile_order: order[N] (host) of bsa_tile_permute's tile order for one
+ *   tile shape; with one shape per head it gives head-aware tilings.
+ *   Errors: BSA_ERR_INVALID_ARG.
+ * bsa_order_tables: from order[n] (host) build the gather tables (host)
+ *   fwd[n_pad] (fwd[p] = order[p] for p < n, -1 for the zero tail) and
+ *   inv[n] (inv[order[p]] = p).  BSA_ERR_INVALID_ARG if order is not a
+ *   permutation of 0..n-1 or n_pad < n.
+ * ------------------------------------------------------------------------- */
+bsa_status bsa_hilbert_order(int T, int Hs, int Ws, int32_t* order);
+bsa_status bsa_tile_order(int T, int Hs, int Ws, int tt, int th, int tw, int32_t* order);
+bsa_status bsa_order_tables(const int32_t* order, int n, int n_pad, int32_t* fwd, int32_t* inv);
+
+/* ---------------------------------------------------------------------------
+ * bsa_gather_rows -- out[b, h, i, :] = in[b, h, src[i], :] on the GPU; a src
+ * entry outside [0, n_in) writes a zero row (the tail pad).
+ *
+ *   in   [B, H, n_in, d] bf16 (any 2-byte rows, moved bit-exactly).
+ *   out  [B, H, n_out, d], must not overlap in.
+ *   src  device int32: [n_out] shared by every head (per_head = 0), or
+ *        [H, n_out], table h for head h of every batch item (per_head = 1).
+ * With fwd from bsa_order_tables (n_out = n_pad) this permutes; with inv
+ * (n_in = n_pad, n_out = n) it restores frame-major order.  d % 8 == 0;
+ * in/out 16-byte aligned, src 4-byte aligned.  Errors: BSA_ERR_INVALID_ARG,
+ * BSA_ERR_UNSUPPORTED (d % 8 != 0), BSA_ERR_OVERFLOW (B*H*max(n_in,
+ * n_out)*d >= 2^40, or per_head with H > 65535), BSA_ERR_MISALIGNED,
+ * BSA_ERR_LAUNCH.  Bit-exact copies.
+ * ------------------------------------------------------------------------- */
+bsa_status bsa_gather_rows(const void* in, void* out, int B, int H, int n_in, int n_out, int d,
+                           const int32_t* src, int per_head, void* stream);
+
+/* ---------------------------------------------------------------------------
  * bsa_forward -- block-sparse attention forward (Sec. 4.3.2: the FlashAttention
  * forward whose key-block loop is replaced by the CRM iterator of Appendix E,
  * Algorithm 2; dense tensor-core work inside each kept tile).

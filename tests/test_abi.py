@@ -90,6 +90,29 @@ def test_threshold_resize_rejects_bad_args(lib):
     assert fn(a, 1 << 20, 4, 4, b, 4096, 8, None) == 4  # H * tq >= 2^31
 
 
+def test_gather_rows_rejects_bad_args(lib):
+    P = ctypes.c_void_p
+    a, b, t = P(0x1000), P(0x2000), P(0x3000)
+    fn = lib.bsa_gather_rows
+    assert fn(None, b, 1, 1, 8, 8, 8, t, 0, None) == 1
+    assert fn(a, b, 1, 1, 8, 8, 8, None, 0, None) == 1
+    assert fn(a, b, 1, 1, 8, 8, 8, t, 2, None) == 1       # per_head must be 0 or 1
+    assert fn(a, b, 1, 1, 0, 8, 8, t, 0, None) == 1
+    assert fn(a, b, 1, 1, 8, 8, 12, t, 0, None) == 2      # d % 8
+    assert fn(P(0x1008), b, 1, 1, 8, 8, 8, t, 0, None) == 3
+    assert fn(a, b, 1, 1, 8, 8, 8, P(0x3002), 0, None) == 3
+    assert fn(a, b, 1, 70000, 8, 8, 8, t, 1, None) == 4   # per-head tables: H <= 65535
+
+
+def test_host_orders_reject_bad_args(lib):
+    P = ctypes.c_void_p
+    buf = (ctypes.c_int32 * 8)()
+    assert lib.bsa_hilbert_order(0, 2, 2, buf) == 1
+    assert lib.bsa_hilbert_order(2, 2, 2, None) == 1
+    assert lib.bsa_tile_order(2, 2, 2, 0, 1, 1, buf) == 1
+    assert lib.bsa_order_tables(buf, 8, 7, buf, buf) == 1  # n_pad < n
+
+
 def test_permute_rejects_bad_args(lib):
     P = ctypes.c_void_p
     a, b = P(0x1000), P(0x2000)
