@@ -28,6 +28,10 @@ Intrinsic Sparse Attention Topology for Video Diffusion Transformers"):
                             Hilbert curve over the enclosing power-of-two cube
                             (Skilling's transpose method), grid points in curve
                             order.
+- ``top_p_mask``         -- online top-p block mask: pooled-query/key block
+                            scores, row softmax, smallest descending prefix
+                            reaching top_p (ScalingAttention Algorithm 1's
+                            sort-and-accumulate cut, per row, per-head top-p).
 """
 from __future__ import annotations
 
@@ -84,6 +88,7 @@ def _load():
             lib.oracle_hilbert_key.restype = ctypes.c_uint64
             lib.oracle_hilbert_order.argtypes = [I, I, I, P]
             lib.oracle_hilbert_order.restype = I
+            lib.oracle_top_p_mask.argtypes = [P, P, I64, I64, I64, I64, I, I, P, P, P, P]
             _lib = lib
     return _lib
 
@@ -224,3 +229,22 @@ def hilbert_order(T: int, Hs: int, Ws: int) -> np.ndarray:
     if _load().oracle_hilbert_order(T, Hs, Ws, _ptr(perm)) < 0:
         raise MemoryError("oracle_hilbert_order")
     return perm
+
+
+def top_p_mask(q_bits, k_bits, H: int, n_valid: int, block: int, tau, top_p,
+               with_prob: bool = False):
+    """q_bits/k_bits raw bf16 [B*H, n_pad, d] in block order; tau, top_p per head [H].
+    Returns mask uint8 [B*H, nb, nb] (and the fp64 probabilities if with_prob)."""
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k_bits = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    BH, n_pad, d = q_bits.shape
+    assert k_bits.shape == q_bits.shape and BH % H == 0
+    nb = n_pad // block
+    tau = np.ascontiguousarray(tau, dtype=np.float64)
+    top_p = np.ascontiguousarray(top_p, dtype=np.float64)
+    assert tau.shape == (H,) and top_p.shape == (H,)
+    mask = np.zeros((BH, nb, nb), dtype=np.uint8)
+    prob = np.zeros((BH, nb, nb), dtype=np.float64) if with_prob else None
+    _load().oracle_top_p_mask(_ptr(q_bits), _ptr(k_bits), BH // H, H, n_valid, n_pad, d, block,
+                              _ptr(tau), _ptr(top_p), _ptr(mask), _ptr(prob))
+    return (mask, prob) if with_prob else mask

@@ -434,3 +434,93 @@ int oracle_hilbert_order(int T, int Hs, int Ws, int64_t* perm) {
   free(tok);
   return bits;
 }
+
+/* ------------------------------------------------------------------ */
+/* Online top-p block mask (dynamic block-sparse prediction).          */
+/*                                                                     */
+/* The block scores and the cut follow ScalingAttention Algorithm 1    */
+/* (sort the block scores, accumulate, cut where the cumulative share  */
+/* reaches p: the Top-k(S, p) of Eq. 2) applied row by row as online   */
+/* top-p predictors do, with a top-p threshold per head (the selective */
+/* head globalization page: per-head top-p thresholds).  The block     */
+/* score is the proxy of pooled queries and keys:                      */
+/*   qbar_i = mean of the valid tokens of query block i, kbar_j alike  */
+/*   s_ij = qbar_i . kbar_j / (sqrt(d) * tau_h),  p_ij = softmax_j s_ij */
+/* Row i keeps the blocks taken in descending p (ties: lower j first)  */
+/* up to and including the one at which the cumulative sum reaches     */
+/* top_p[h] (at least one block; all blocks if the sum never does).    */
+/*   q, k   raw bf16 [B*H, n_pad, d] (tokens in block order)           */
+/*   mask   out uint8 [B*H, nb, nb];  prob out double [B*H, nb, nb]    */
+/*          (may be NULL)                                              */
+/* ------------------------------------------------------------------ */
+typedef struct {
+  double p;
+  int j;
+} prob_entry;
+
+static int cmp_prob_desc(const void* pa, const void* pb) {
+  const prob_entry* a = (const prob_entry*)pa;
+  const prob_entry* b = (const prob_entry*)pb;
+  if (a->p > b->p) return -1;
+  if (a->p < b->p) return 1;
+  return (a->j > b->j) - (a->j < b->j);
+}
+
+static void block_means(const uint16_t* x, int64_t n_valid, int d, int block, int nb,
+                        double* out /* [nb, d] */) {
+  for (int i = 0; i < nb; ++i) {
+    int64_t lo = (int64_t)i * block, hi = lo + block;
+    if (hi > n_valid) hi = n_valid;
+    for (int c = 0; c < d; ++c) out[(int64_t)i * d + c] = 0.0;
+    for (int64_t t = lo; t < hi; ++t)
+      for (int c = 0; c < d; ++c) out[(int64_t)i * d + c] += bf16_bits_to_double(x[t * d + c]);
+    const double cnt = (double)(hi - lo);
+    for (int c = 0; c < d; ++c) out[(int64_t)i * d + c] /= cnt;
+  }
+}
+
+void oracle_top_p_mask(const uint16_t* q, const uint16_t* k, int64_t B, int64_t H,
+                       int64_t n_valid, int64_t n_pad, int d, int block, const double* tau,
+                       const double* top_p, uint8_t* mask, double* prob) {
+  const int nb = (int)(n_pad / block);
+#pragma omp parallel for schedule(dynamic)
+  for (int64_t bh = 0; bh < B * H; ++bh) {
+    const int64_t h = bh % H;
+    double* qm = (double*)malloc(sizeof(double) * (size_t)nb * d);
+    double* km = (double*)malloc(sizeof(double) * (size_t)nb * d);
+    double* s = (double*)malloc(sizeof(double) * (size_t)nb);
+    prob_entry* order = (prob_entry*)malloc(sizeof(prob_entry) * (size_t)nb);
+    block_means(q + bh * n_pad * d, n_valid, d, block, nb, qm);
+    block_means(k + bh * n_pad * d, n_valid, d, block, nb, km);
+    const double denom = sqrt((double)d) * tau[h];
+    for (int i = 0; i < nb; ++i) {
+      double m = -INFINITY;
+      for (int j = 0; j < nb; ++j) {
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += qm[(int64_t)i * d + c] * km[(int64_t)j * d + c];
+        s[j] = dot / denom;
+        if (s[j] > m) m = s[j];
+      }
+      double l = 0.0;
+      for (int j = 0; j < nb; ++j) l += exp(s[j] - m);
+      uint8_t* row = mask + (bh * nb + i) * (int64_t)nb;
+      for (int j = 0; j < nb; ++j) {
+        order[j].p = exp(s[j] - m) / l;
+        order[j].j = j;
+        row[j] = 0;
+        if (prob) prob[(bh * nb + i) * (int64_t)nb + j] = order[j].p;
+      }
+      qsort(order, (size_t)nb, sizeof(prob_entry), cmp_prob_desc);
+      double cum = 0.0;
+      for (int r = 0; r < nb; ++r) {
+        row[order[r].j] = 1;
+        cum += order[r].p;
+        if (cum >= top_p[h]) break;
+      }
+    }
+    free(qm);
+    free(km);
+    free(s);
+    free(order);
+  }
+}
