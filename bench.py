@@ -18,8 +18,9 @@ max over ranks.
 
 After the timed steps, `next_rows` reports further steps measured on their own
 (L2 flushed before each call): bsa_pack_mask_from_threshold at the workload's
-block grid, bsa_threshold_resize of a 480p-grid map to it, and bsa_gather_rows
-applying the Hilbert-curve order and head-aware tile orders to one tensor.
+block grid, bsa_threshold_resize of a 480p-grid map to it, bsa_gather_rows
+applying the Hilbert-curve order and head-aware tile orders to one tensor, and
+the online top-p predictor bsa_predict_top_p on the workload's q and k.
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of query blocks of the same workload (rank 0 only).
@@ -323,6 +324,36 @@ def measure_order_rows(w, dev, stream, hbm_gbs: float):
     return res
 
 
+def measure_predict_row(w, dev, stream, hbm_gbs: float):
+    """bsa_predict_top_p on the workload's block-ordered q and k (synthetic
+    per-head tau and top_p).  Roofline: HBM, algorithmic bytes = q and k read
+    once (the pooled means, 24 MB at 720p, and the mask outputs are counted
+    too)."""
+    import block_sparse_attention_forward_b200 as bsa
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    q, k, _ = I.gen_qkv(w, seed=w.seed + 5000)
+    grid, tile = (w.T, w.Hs, w.Ws), (w.tt, w.th, w.tw)
+    qp = bsa.tile_permute(q.to(dev), grid, tile, w.n_pad)
+    kp = bsa.tile_permute(k.to(dev), grid, tile, w.n_pad)
+    del q, k
+    tau, top_p = I.gen_top_p_params(w)
+    tau_d, top_d = torch.from_numpy(tau).to(dev), torch.from_numpy(top_p).to(dev)
+    pm = bsa.predict_top_p(qp, kp, w.n, w.block, tau_d, top_d)
+    torch.cuda.synchronize(dev)
+    rows = w.B * w.H * w.nb
+    kept = int(pm.row_offsets[-1])
+    words = (w.nb + 31) // 32
+    nbytes = (2 * w.B * w.H * w.n * w.d * 2 + 2 * rows * w.d * 4
+              + 4 * (rows * words + 3 * rows + 1 + kept))
+    us = time_device_us(lambda: bsa.predict_top_p(qp, kp, w.n, w.block, tau_d, top_d), stream,
+                        flush)
+    gbs = nbytes / (us * 1e-6) / 1e9
+    del flush, qp, kp
+    return {"predict_top_p": {"us": us, "bytes": nbytes, "achieved_gbs": gbs,
+                              "frac_hbm": gbs / hbm_gbs, "bound": "hbm", "launches": 6,
+                              "density": kept / (rows * w.nb), "l2": "flushed before each call"}}
+
+
 def workload_config(w, mask):
     kept = I.kept_tiles(mask)
     total = w.B * w.H * w.nb * w.nb
@@ -368,6 +399,8 @@ def main():
                                       float(peaks["hbm_gbs"]))
         rows.update(measure_order_rows(w, dev, torch.cuda.current_stream(dev),
                                        float(peaks["hbm_gbs"])))
+        rows.update(measure_predict_row(w, dev, torch.cuda.current_stream(dev),
+                                        float(peaks["hbm_gbs"])))
         if rank == 0:
             print(json.dumps({"workload": w.name, "next_rows": rows}), flush=True)
         if world > 1:
@@ -492,6 +525,7 @@ def main():
     if not args.no_next:
         next_rows = measure_threshold_rows(w, dev, stream, float(peaks["hbm_gbs"]))
         next_rows.update(measure_order_rows(w, dev, stream, float(peaks["hbm_gbs"])))
+        next_rows.update(measure_predict_row(w, dev, stream, float(peaks["hbm_gbs"])))
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",

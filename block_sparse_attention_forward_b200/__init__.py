@@ -27,7 +27,7 @@ from . import _ffi
 from ._ffi import BsaError, BsaMask
 
 __all__ = ["BsaError", "PackedMask", "pack_mask", "pack_mask_from_threshold",
-           "threshold_resize", "tile_permute", "tile_unpermute", "hilbert_order", "tile_order",
+           "threshold_resize", "predict_top_p", "tile_permute", "tile_unpermute", "hilbert_order", "tile_order",
            "order_tables", "gather_rows", "forward", "device_error", "version"]
 
 
@@ -182,6 +182,31 @@ def tile_unpermute(y: torch.Tensor, grid, tile, out: torch.Tensor | None = None)
                                         tw, n_pad, _stream(y.device))
     _ffi.check(st, "bsa_tile_unpermute")
     return out
+
+
+def predict_top_p(q: torch.Tensor, k: torch.Tensor, n_valid: int, block: int,
+                  tau: torch.Tensor, top_p: torch.Tensor, with_lists: bool = True) -> PackedMask:
+    """Online top-p block mask of block-ordered q, k [B, H, n_pad, d] bf16 with
+    per-head tau and top_p (fp32 [H] on the GPU) -> PackedMask (bsa_predict_top_p)."""
+    _require_cuda(q, "q", torch.bfloat16)
+    _require_cuda(k, "k", torch.bfloat16)
+    _require_cuda(tau, "tau", torch.float32)
+    _require_cuda(top_p, "top_p", torch.float32)
+    B, H, n_pad, d = q.shape
+    if k.shape != q.shape:
+        raise ValueError("q and k shapes differ")
+    if tau.shape != (H,) or top_p.shape != (H,):
+        raise ValueError("tau and top_p must be [H]")
+    nb = n_pad // block
+    lib = _ffi.load()
+    pm = _packed_outputs(B, H, nb, nb, q.device, with_lists)
+    ws_bytes = lib.bsa_predict_top_p_workspace(B, H, n_pad, d, block)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    st = lib.bsa_predict_top_p(q.data_ptr(), k.data_ptr(), B, H, int(n_valid), n_pad, d,
+                               int(block), tau.data_ptr(), top_p.data_ptr(), *_pack_pointers(pm),
+                               ws.data_ptr(), ws.numel(), _stream(q.device))
+    _ffi.check(st, "bsa_predict_top_p")
+    return pm
 
 
 def _host_i32(n: int) -> torch.Tensor:

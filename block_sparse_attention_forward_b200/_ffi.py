@@ -31,6 +31,8 @@ EXPORTED = (
     "bsa_pack_mask_noalloc",
     "bsa_pack_mask_from_threshold",
     "bsa_threshold_resize",
+    "bsa_predict_top_p_workspace",
+    "bsa_predict_top_p",
     "bsa_hilbert_order",
     "bsa_tile_order",
     "bsa_order_tables",
@@ -90,6 +92,10 @@ def load() -> ctypes.CDLL:
     lib.bsa_pack_mask_from_threshold.restype = I
     lib.bsa_threshold_resize.argtypes = [P, I, I, I, P, I, I, P]
     lib.bsa_threshold_resize.restype = I
+    lib.bsa_predict_top_p_workspace.argtypes = [I, I, I, I, I]
+    lib.bsa_predict_top_p_workspace.restype = SZ
+    lib.bsa_predict_top_p.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P, P, P, P, P, SZ, P]
+    lib.bsa_predict_top_p.restype = I
     lib.bsa_hilbert_order.argtypes = [I, I, I, P]
     lib.bsa_hilbert_order.restype = I
     lib.bsa_tile_order.argtypes = [I, I, I, I, I, I, P]

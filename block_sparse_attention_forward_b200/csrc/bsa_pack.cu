@@ -403,11 +403,23 @@ bsa_status launch_offsets_schedule_lists(const uint32_t* bits, const int32_t* co
 
 }  // namespace
 
+static_assert(bsa::kPackMaxNbK + 1 == kMaxBins, "packing limit");
+
+size_t bsa::pack_scratch_bytes(int64_t rows, int nb_k) {
+  const size_t bytes = size_t(workspace_ints(rows, nb_k)) * sizeof(int32_t);
+  return (bytes + 255) & ~size_t(255);
+}
+
+bsa_status bsa::pack_finish(const uint32_t* bits, const int32_t* counts, int rows, int nb_k,
+                            int32_t* row_offsets, int32_t* col_idx, int32_t* schedule,
+                            void* scratch, cudaStream_t s) {
+  return launch_offsets_schedule_lists(bits, counts, rows, nb_k, (nb_k + 31) / 32, row_offsets,
+                                       col_idx, schedule, static_cast<int32_t*>(scratch), s);
+}
+
 extern "C" size_t bsa_pack_mask_workspace(int B, int H, int nb_q, int nb_k) {
   if (B <= 0 || H <= 0 || nb_q <= 0 || nb_k <= 0) return 0;
-  const size_t bytes =
-      size_t(workspace_ints(int64_t(B) * H * nb_q, nb_k)) * sizeof(int32_t);
-  return (bytes + 255) & ~size_t(255);
+  return bsa::pack_scratch_bytes(int64_t(B) * H * nb_q, nb_k);
 }
 
 extern "C" bsa_status bsa_pack_mask(const uint8_t* dense, int B, int H, int nb_q, int nb_k,

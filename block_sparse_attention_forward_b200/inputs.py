@@ -293,6 +293,21 @@ def gen_threshold(w: Workload, seed: int | None = None):
     return thr, p
 
 
+def gen_top_p_params(w: Workload, seed: int | None = None):
+    """Per-head temperature and top-p threshold for the online top-p predictor.
+
+    The pooled-query/key score of N(0,1) tokens scales like 1 / (block * tau),
+    so tau_h = c_h / block with c_h log-uniform on [0.35, 0.7] gives masks of
+    roughly 15-40 % density; top_p_h ~ U[0.85, 0.95] (per-head top-p
+    thresholds).  Returns (tau float32 [H], top_p float32 [H])."""
+    seed = (w.seed if seed is None else seed) + 4000
+    rng = np.random.default_rng(seed)
+    c = np.exp(rng.uniform(np.log(0.35), np.log(0.7), size=w.H))
+    tau = (c / w.block).astype(np.float32)
+    top_p = rng.uniform(0.85, 0.95, size=w.H).astype(np.float32)
+    return tau, top_p
+
+
 def kept_tiles(mask: np.ndarray) -> int:
     return int(np.count_nonzero(mask))
 

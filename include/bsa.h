@@ -208,6 +208,41 @@ bsa_status bsa_tile_unpermute(const void* in, void* out, int B, int H, int T, in
                               int d, int tt, int th, int tw, int n_pad, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * bsa_predict_top_p -- online top-p block mask from the (permuted) q and k,
+ * straight to the CRM rows, lists and schedule that bsa_forward reads.
+ *
+ * The cut follows Algorithm 1 (sort the block scores, accumulate, cut where
+ * the cumulative share reaches p: Top-k(S, p) of Eq. 2), applied per query
+ * block with one top-p threshold per head, on the proxy scores of pooled
+ * queries and keys:
+ *   qbar_i = mean of the valid tokens of block i (kbar_j alike)
+ *   s_ij = qbar_i . kbar_j / (sqrt(d) * tau[h]),  p_ij = softmax_j(s_ij)
+ * Row i keeps the blocks in descending p (ties: lower j first) up to and
+ * including the one where the cumulative sum reaches top_p[h]; at least one
+ * block, all of them if the sum never reaches it.  Arithmetic: fp32 means,
+ * fp32 FMA scores, expf; the cumulative comparison is in fp32, so a block whose
+ * inclusion changes the sum by less than fp32 rounding can go either way.
+ *
+ *   q, k      [B, H, n_pad, d] bf16 in block order (as given to bsa_forward).
+ *   tau, top_p  [H] fp32 device arrays.
+ *   bits, counts, row_offsets, col_idx, schedule: as for bsa_pack_mask with
+ *             nb_q = nb_k = n_pad / block.
+ *   workspace device scratch of bsa_predict_top_p_workspace(...) bytes,
+ *             16-byte aligned (pooled means and the sort's tables).
+ *
+ * Supported: d in {64, 128}; n_pad % block == 0; n_pad - block < n_valid <=
+ * n_pad; n_pad / block <= 2048; B*H <= 65535.  Errors: BSA_ERR_INVALID_ARG,
+ * BSA_ERR_UNSUPPORTED, BSA_ERR_OVERFLOW, BSA_ERR_MISALIGNED (q, k,
+ * workspace 16-byte; others 4-byte), BSA_ERR_WORKSPACE, BSA_ERR_LAUNCH.
+ * ------------------------------------------------------------------------- */
+size_t bsa_predict_top_p_workspace(int B, int H, int n_pad, int d, int block);
+bsa_status bsa_predict_top_p(const void* q, const void* k, int B, int H, int n_valid, int n_pad,
+                             int d, int block, const float* tau, const float* top_p,
+                             uint32_t* bits, int32_t* counts, int32_t* row_offsets,
+                             int32_t* col_idx, int32_t* schedule, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Token orders as tables, and the gather that applies them.
  *
  * Token permutation eases the 128 x 128 granularity bottleneck by clustering
