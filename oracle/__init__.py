@@ -18,7 +18,9 @@ Intrinsic Sparse Attention Topology for Video Diffusion Transformers"):
 - ``tile_order``, ``permute``, ``unpermute``
                          -- token reordering into 3-D tiles, Sec. 5.4 and 5.5.
 - ``attention``          -- Sec. 4.3.2 block-sparse FlashAttention forward,
-                            written as plain masked softmax attention in fp64.
+                            written as plain masked softmax attention in fp64;
+                            query and key blocks may differ in size (finer key
+                            blocks: Sec. 5.4, the granularity bottleneck).
 - ``threshold_mask``     -- Sec. 4.1.2 (Eq. 2, M_p = 1(T <= p)) with one
                             threshold per head (Algorithm 1, FAST).
 - ``threshold_resize``   -- Sec. 4.3.1, Eq. 7 (conservative bilinear resize of
@@ -82,6 +84,8 @@ def _load():
             lib.oracle_unpermute.argtypes = [P, P, I64, I64, I64, I, P]
             lib.oracle_attention.argtypes = [P, P, P, P, I64, I64, I64, I, I, ctypes.c_double,
                                              P, I64, I, P, P]
+            lib.oracle_attention_blocks.argtypes = [P, P, P, P, I64, I64, I64, I, I, I,
+                                                    ctypes.c_double, P, I64, I, P, P]
             lib.oracle_threshold_mask.argtypes = [P, P, I, I, I, I, P]
             lib.oracle_threshold_resize.argtypes = [P, I, I, I, P, I, I]
             lib.oracle_hilbert_key.argtypes = [I, I, I, I]
@@ -168,10 +172,12 @@ def unpermute(y_bits: np.ndarray, perm: np.ndarray, n: int) -> np.ndarray:
 
 
 def attention(q_bits, k_bits, v_bits, mask, n_valid: int, block: int, scale: float | None = None,
-              rows: np.ndarray | None = None, dense_literal: bool = False):
+              rows: np.ndarray | None = None, dense_literal: bool = False,
+              block_k: int | None = None):
     """Masked softmax attention in fp64 over permuted tokens.
 
-    q_bits/k_bits/v_bits: uint16 raw bf16, [BH, n_pad, d].  mask: uint8 [BH, nb, nb].
+    q_bits/k_bits/v_bits: uint16 raw bf16, [BH, n_pad, d].  mask: uint8
+    [BH, n_pad // block, n_pad // block_k] (block_k defaults to block).
     rows: optional int64 flat query ids (bh * n_pad + i).  Returns (out [R, d], lse [R])
     in float64, R = len(rows) or BH * n_pad.
     """
@@ -191,9 +197,11 @@ def attention(q_bits, k_bits, v_bits, mask, n_valid: int, block: int, scale: flo
         rows_p = _ptr(rows)
     out = np.zeros((n_rows, d), dtype=np.float64)
     lse = np.zeros(n_rows, dtype=np.float64)
-    _load().oracle_attention(_ptr(q_bits), _ptr(k_bits), _ptr(v_bits), _ptr(mask), BH, n_valid,
-                             n_pad, d, block, float(scale), rows_p, n_rows, int(dense_literal),
-                             _ptr(out), _ptr(lse))
+    block_k = block if block_k is None else int(block_k)
+    assert mask.shape == (BH, n_pad // block, n_pad // block_k), mask.shape
+    _load().oracle_attention_blocks(_ptr(q_bits), _ptr(k_bits), _ptr(v_bits), _ptr(mask), BH,
+                                    n_valid, n_pad, d, block, block_k, float(scale), rows_p,
+                                    n_rows, int(dense_literal), _ptr(out), _ptr(lse))
     return out, lse
 
 

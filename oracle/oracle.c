@@ -217,11 +217,18 @@ void oracle_unpermute(const uint16_t* in, uint16_t* out, int64_t BH, int64_t n, 
 /* Outputs: out [n_rows, d], lse [n_rows].  Rows with no valid kept key */
 /* and pad rows (i >= n_valid) give out = 0, lse = -inf.                */
 /* ------------------------------------------------------------------ */
-void oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                      const uint8_t* mask, int64_t BH, int64_t n_valid, int64_t n_pad, int d,
-                      int block, double scale, const int64_t* rows, int64_t n_rows,
-                      int dense_literal, double* out, double* lse) {
-  const int64_t nb = n_pad / block;
+/* Query blocks of block_q tokens and key blocks of block_k tokens: the mask is
+ * [BH, n_pad / block_q, n_pad / block_k] and query i, key j are in blocks
+ * i / block_q and j / block_k.  (Equal sizes are the method as the pages run
+ * it; block_k = block_q / 2 is the finer key granularity they name as the
+ * remedy for the 128 x 128 granularity bottleneck.) */
+void oracle_attention_blocks(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             const uint8_t* mask, int64_t BH, int64_t n_valid, int64_t n_pad,
+                             int d, int block_q, int block_k, double scale, const int64_t* rows,
+                             int64_t n_rows, int dense_literal, double* out, double* lse) {
+  const int64_t nb_q = n_pad / block_q, nb_k = n_pad / block_k;
+  (void)nb_q;
+  const int block = block_k; /* the key-side block, as the loops below walk keys */
   if (rows == NULL) n_rows = BH * n_pad;
 
 #pragma omp parallel
@@ -239,7 +246,7 @@ void oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
 
       const uint16_t* qrow = q + (bh * n_pad + i) * d;
       for (int c = 0; c < d; ++c) qi[c] = bf16_bits_to_double(qrow[c]);
-      const uint8_t* mrow = mask + (bh * nb + i / block) * nb;
+      const uint8_t* mrow = mask + (bh * nb_q + i / block_q) * nb_k;
 
       /* scores s_j for j < n_valid; -inf where the key block is masked */
       double m = -INFINITY;
@@ -276,6 +283,15 @@ void oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     free(s);
     free(qi);
   }
+}
+
+/* One block size for queries and keys (mask [BH, nb, nb]). */
+void oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                      const uint8_t* mask, int64_t BH, int64_t n_valid, int64_t n_pad, int d,
+                      int block, double scale, const int64_t* rows, int64_t n_rows,
+                      int dense_literal, double* out, double* lse) {
+  oracle_attention_blocks(q, k, v, mask, BH, n_valid, n_pad, d, block, block, scale, rows, n_rows,
+                          dense_literal, out, lse);
 }
 
 /* ------------------------------------------------------------------ */
