@@ -19,8 +19,9 @@ max over ranks.
 After the timed steps, `next_rows` reports further steps measured on their own
 (L2 flushed before each call): bsa_pack_mask_from_threshold at the workload's
 block grid, bsa_threshold_resize of a 480p-grid map to it, bsa_gather_rows
-applying the Hilbert-curve order and head-aware tile orders to one tensor, and
-the online top-p predictor bsa_predict_top_p on the workload's q and k.
+applying the Hilbert-curve order and head-aware tile orders to one tensor,
+the online top-p predictor bsa_predict_top_p on the workload's q and k, and the
+forward with 64-token key blocks under 128-token query blocks.
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of query blocks of the same workload (rank 0 only).
@@ -354,6 +355,38 @@ def measure_predict_row(w, dev, stream, hbm_gbs: float):
                               "density": kept / (rows * w.nb), "l2": "flushed before each call"}}
 
 
+def measure_finer_keys_row(w, dev, stream, peak_tflops: float):
+    """bsa_forward_blocks with 128-token query blocks over 64-token key blocks on
+    the workload (mask from inputs.gen_mask_fine).  Roofline: tensor; algorithmic
+    work 4 * d * 128 * 64 FLOP per kept (query block, key block) pair."""
+    import block_sparse_attention_forward_b200 as bsa
+    if w.block != 128 or (w.n_pad - w.n) >= 64:
+        return {"forward_finer_keys": None}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    q, k, v = I.gen_qkv(w, seed=w.seed + 7000)
+    mask = I.gen_mask_fine(w, seed=w.seed + 7000)
+    grid, tile = (w.T, w.Hs, w.Ws), (w.tt, w.th, w.tw)
+    qp, kp, vp = (bsa.tile_permute(t.to(dev), grid, tile, w.n_pad) for t in (q, k, v))
+    del q, k, v
+    pm = bsa.pack_mask(torch.from_numpy(mask).to(dev))
+    out = torch.empty_like(qp)
+    lse = torch.empty((w.B, w.H, w.n_pad), dtype=torch.float32, device=dev)
+    kept = I.kept_tiles(mask)
+    flops = 4.0 * w.d * w.block * (w.block // 2) * kept
+    us = time_device_us(lambda: bsa.forward(qp, kp, vp, pm, w.n, w.block, out=out, lse=lse,
+                                            block_k=w.block // 2), stream, flush, iters=5,
+                        warmup=3)
+    if bsa.device_error() != 0:
+        raise RuntimeError("device error in the finer-key forward")
+    tf = flops / (us * 1e-6) / 1e12
+    del flush, qp, kp, vp, out
+    return {"forward_finer_keys": {"block_q": w.block, "block_k": w.block // 2, "us": us,
+                                   "kept_pairs": kept,
+                                   "density": kept / (w.B * w.H * w.nb * 2 * w.nb),
+                                   "achieved_tflops": tf, "peak": peak_tflops,
+                                   "frac": tf / peak_tflops, "bound": "tensor", "launches": 1}}
+
+
 def workload_config(w, mask):
     kept = I.kept_tiles(mask)
     total = w.B * w.H * w.nb * w.nb
@@ -401,6 +434,9 @@ def main():
                                        float(peaks["hbm_gbs"])))
         rows.update(measure_predict_row(w, dev, torch.cuda.current_stream(dev),
                                         float(peaks["hbm_gbs"])))
+        rows.update(measure_finer_keys_row(w, dev, torch.cuda.current_stream(dev),
+                                           float(peaks.get("bf16_tflops_sustained",
+                                                           peaks.get("bf16_tflops")))))
         if rank == 0:
             print(json.dumps({"workload": w.name, "next_rows": rows}), flush=True)
         if world > 1:
@@ -521,16 +557,17 @@ def main():
 
     # ---------------------------------------------------------------- roofline
     peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     next_rows = None
     if not args.no_next:
         next_rows = measure_threshold_rows(w, dev, stream, float(peaks["hbm_gbs"]))
         next_rows.update(measure_order_rows(w, dev, stream, float(peaks["hbm_gbs"])))
         next_rows.update(measure_predict_row(w, dev, stream, float(peaks["hbm_gbs"])))
-    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        next_rows.update(measure_finer_keys_row(w, dev, stream, peak))
     fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
                 "frac": fwd_tflops / peak, "traffic": recorded_traffic(w.name),
-                "kernel": "bsa_forward_kernel<128,128>",
+                "kernel": "bsa_forward_kernel<128,128,128>",
                 "peak_source": f"{peak_src} bf16_tflops_sustained (dense bf16 cuBLAS, seconds-long loop)",
                 "fwd_ms": fwd_ms}
 

@@ -268,8 +268,9 @@ def gather_rows(x: torch.Tensor, src: torch.Tensor, n_out: int | None = None,
 
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask: PackedMask, n_valid: int,
             block: int, softmax_scale: float | None = None, out: torch.Tensor | None = None,
-            lse: torch.Tensor | None = None):
-    """Block-sparse attention forward (bsa_forward) on tile-major q, k, v [B, H, n_pad, d] bf16.
+            lse: torch.Tensor | None = None, block_k: int | None = None):
+    """Block-sparse attention forward (bsa_forward, or bsa_forward_blocks when
+    block_k differs from block) on tile-major q, k, v [B, H, n_pad, d] bf16.
 
     Returns (out bf16 [B, H, n_pad, d], lse fp32 [B, H, n_pad])."""
     for t, name in ((q, "q"), (k, "k"), (v, "v")):
@@ -284,10 +285,18 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask: PackedMask,
     _require_cuda(out, "out", torch.bfloat16)
     _require_cuda(lse, "lse", torch.float32)
     cm = mask.as_c()
-    st = _ffi.load().bsa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(cm),
-                                 out.data_ptr(), lse.data_ptr(), B, H, int(n_valid), n_pad, d,
-                                 int(block), float(softmax_scale or 0.0), _stream(q.device))
-    _ffi.check(st, "bsa_forward")
+    lib = _ffi.load()
+    if block_k is None or int(block_k) == int(block):
+        st = lib.bsa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(cm),
+                             out.data_ptr(), lse.data_ptr(), B, H, int(n_valid), n_pad, d,
+                             int(block), float(softmax_scale or 0.0), _stream(q.device))
+        _ffi.check(st, "bsa_forward")
+    else:
+        st = lib.bsa_forward_blocks(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(cm),
+                                    out.data_ptr(), lse.data_ptr(), B, H, int(n_valid), n_pad, d,
+                                    int(block), int(block_k), float(softmax_scale or 0.0),
+                                    _stream(q.device))
+        _ffi.check(st, "bsa_forward_blocks")
     return out, lse
 
 

@@ -40,6 +40,7 @@ EXPORTED = (
     "bsa_tile_permute",
     "bsa_tile_unpermute",
     "bsa_forward",
+    "bsa_forward_blocks",
     "bsa_get_device_error",
 )
 
@@ -111,6 +112,9 @@ def load() -> ctypes.CDLL:
     lib.bsa_forward.argtypes = [P, P, P, ctypes.POINTER(BsaMask), P, P, I, I, I, I, I, I,
                                 ctypes.c_float, P]
     lib.bsa_forward.restype = I
+    lib.bsa_forward_blocks.argtypes = [P, P, P, ctypes.POINTER(BsaMask), P, P, I, I, I, I, I, I,
+                                       I, ctypes.c_float, P]
+    lib.bsa_forward_blocks.restype = I
     lib.bsa_get_device_error.argtypes = [ctypes.POINTER(I)]
     lib.bsa_get_device_error.restype = I
     _lib = lib

@@ -24,9 +24,12 @@
 //     while the softmax works on S(n).
 //   * work order: query tiles are taken from the count-descending schedule
 //     (heaviest first), CTA c handles tiles c, c + grid, ...
-//   * a tile is always 128 query rows; with 64-token blocks it holds two query
-//     blocks and walks the union of their CRM rows, each row masking the key
-//     blocks its own query block did not keep.
+//   * a tile is always 128 query rows; with 64-token query blocks it holds two
+//     query blocks and walks the union of their CRM rows, each row masking the
+//     key blocks its own query block did not keep.  Key blocks may be smaller
+//     than query blocks (128-row query blocks over 64-key blocks: twice the
+//     CRM bits per row, the finer key granularity Sec. 5.4 asks for below 40 %
+//     density); a kept key block is then an M = 128, N = 64 product.
 //   * every barrier wait is bounded (about two seconds); a wait that runs out
 //     records BSA_ERR_TIMEOUT in a device word, the CTA drains what it has in
 //     flight and exits.
@@ -57,19 +60,19 @@ constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
 struct FwdParams {
   const __nv_bfloat16* q;   // [BH, n_pad, d]
   const uint32_t* bits;     // [BH, nb, words]
-  const int32_t* schedule;  // [BH * nb] (used when one query block per tile)
+  const int32_t* schedule;  // [BH * nb_q] (used when one query block per tile)
   __nv_bfloat16* out;       // [BH, n_pad, d]
   float* lse;               // [BH, n_pad]
-  int BH, nb, words, n_valid, n_pad;
+  int BH, nb_q, nb_k, words, n_valid, n_pad;
   int num_tiles, tiles_per_head;
   float scale_log2;
 };
 
-template <int D, int BLK>
+template <int D, int BQ, int BK>
 struct Cfg {
-  static constexpr int R = kTileM / BLK;                        // query blocks per tile
+  static constexpr int R = kTileM / BQ;                         // query blocks per tile
   static constexpr int kRegions = D / 64;                       // 128-byte column groups
-  static constexpr uint32_t kKVRegion = BLK * 128;
+  static constexpr uint32_t kKVRegion = BK * 128;
   static constexpr uint32_t kSlotBytes = kRegions * kKVRegion;  // one K or V tile
   static constexpr uint32_t kMaxSmem = 227u * 1024u;
   static constexpr int kFitStages = int((kMaxSmem - 256 - 1024) / kSlotBytes);
@@ -80,7 +83,7 @@ struct Cfg {
   // fits on the SM (each CTA owns all 512 TMEM columns)
   static constexpr uint32_t kSmemUsed = kOffBar + 256 + 1024;
   static constexpr uint32_t kSmemBytes = kSmemUsed > 120u * 1024u ? kSmemUsed : 120u * 1024u;
-  static constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, BLK, false);
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, BK, false);
   static_assert(kSmemUsed <= kMaxSmem, "shared memory budget");
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, true);
 };
@@ -162,14 +165,14 @@ __device__ __forceinline__ TileInfo tile_info(const FwdParams& p, int tile) {
   TileInfo t;
   if (R == 1) {
     const int row = __ldg(p.schedule + tile);
-    t.bh = row / p.nb;
-    t.qb0 = row - t.bh * p.nb;
+    t.bh = row / p.nb_q;
+    t.qb0 = row - t.bh * p.nb_q;
   } else {
     t.bh = tile / p.tiles_per_head;
     t.qb0 = (tile - t.bh * p.tiles_per_head) * R;
   }
-  t.row0 = p.bits + (int64_t(t.bh) * p.nb + t.qb0) * p.words;
-  t.row1 = (R > 1 && t.qb0 + 1 < p.nb) ? t.row0 + p.words : nullptr;
+  t.row0 = p.bits + (int64_t(t.bh) * p.nb_q + t.qb0) * p.words;
+  t.row1 = (R > 1 && t.qb0 + 1 < p.nb_q) ? t.row0 + p.words : nullptr;
   return t;
 }
 
@@ -180,11 +183,11 @@ __device__ __forceinline__ int union_count(const TileInfo& t, int words) {
   return c;
 }
 
-template <int D, int BLK>
+template <int D, int BQ, int BK>
 __global__ void __launch_bounds__(kThreads, 1)
     bsa_forward_kernel(const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using C = Cfg<D, BLK>;
+  using C = Cfg<D, BQ, BK>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 128-byte swizzle atoms need 1024-byte aligned shared-memory tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -234,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         CrmIter it;
         it.init(t.row0, t.row1, p.words);
         for (int j = it.index(); j >= 0; it.next(), j = it.index()) {
-          const int32_t kv_row = t.bh * p.n_pad + j * BLK;
+          const int32_t kv_row = t.bh * p.n_pad + j * BK;
 #pragma unroll
           for (int kv = 0; kv < 2; ++kv) {  // K then V
             const uint32_t slot = item % C::kStages;
@@ -280,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // keys (2048 bytes) per step
         const uint32_t v_base = sKV + slot * C::kSlotBytes;
 #pragma unroll
-        for (int kk = 0; kk < BLK / 16; ++kk) {
+        for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t bdesc = smem_desc_sw128(v_base + kk * 16 * 128, C::kKVRegion, 1024);
           mma_ts(tmem + kTmemO, p_tmem + kk * 8, bdesc, C::kIdescPV, (first && kk == 0) ? 0u : 1u);
         }
@@ -344,10 +347,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool has_tail = p.n_valid < p.n_pad;
     for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
       const TileInfo t = tile_info<C::R>(p, tile);
-      const int my_qb = t.qb0 + row / BLK;
-      const bool row_in_head = my_qb < p.nb;
-      const uint32_t* my_bits = p.bits + (int64_t(t.bh) * p.nb + my_qb) * p.words;
-      const int64_t tok = int64_t(t.qb0) * BLK + row;  // token index inside the head
+      const int my_qb = t.qb0 + row / BQ;
+      const bool row_in_head = my_qb < p.nb_q;
+      const uint32_t* my_bits = p.bits + (int64_t(t.bh) * p.nb_q + my_qb) * p.words;
+      const int64_t tok = int64_t(t.qb0) * BQ + row;  // token index inside the head
       float m_run = -INFINITY, l_run = 0.0f;
 
       if (union_count(t, p.words) > 0) {
@@ -389,22 +392,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t s_tmem = tmem + lane_base + (sb ? kTmemS1 : kTmemS0);
-        uint32_t sr[BLK];  // raw fp32 scores of this row, one tcgen05.ld
-        if constexpr (BLK == 128) tmem_load128(s_tmem, sr);
+        uint32_t sr[BK];  // raw fp32 scores of this row, one tcgen05.ld
+        if constexpr (BK == 128) tmem_load128(s_tmem, sr);
         else tmem_load64(s_tmem, sr);
         bool member = row_in_head;
         if (C::R > 1 && member) member = (__ldg(my_bits + (j >> 5)) >> (j & 31)) & 1u;
-        if (has_tail && j == p.nb - 1) {
-          const int valid = p.n_valid - j * BLK;
+        if (has_tail && j == p.nb_k - 1) {
+          const int valid = p.n_valid - j * BK;
 #pragma unroll
-          for (int c = 0; c < BLK; ++c)
+          for (int c = 0; c < BK; ++c)
             if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
         }
         float mx8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(sr[i]);
 #pragma unroll
-        for (int c = 8; c < BLK; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+        for (int c = 8; c < BK; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         // Lazy rescale: the reference max only moves when the row max grows by
@@ -447,9 +450,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) sum8[i] = 0.0f;
         const float neg_m = -m_new;
-        uint32_t pk[BLK / 2];
+        uint32_t pk[BK / 2];
 #pragma unroll
-        for (int i = 0; i < BLK / 2; ++i) {
+        for (int i = 0; i < BK / 2; ++i) {
           float p0 = 0.0f, p1 = 0.0f;
           if (member) {
             p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), p.scale_log2, neg_m));
@@ -461,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // P overwrites the first half of this S buffer: packed bf16 pairs, one
         // 32-bit column per two keys
-        if constexpr (BLK == 128) tmem_store64(s_tmem, pk);
+        if constexpr (BK == 128) tmem_store64(s_tmem, pk);
         else tmem_store32(s_tmem, pk);
         const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
                           ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
@@ -565,14 +568,14 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int d, int box_r
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BLK>
+template <int D, int BQ, int BK>
 bsa_status launch_forward(const void* q, const void* k, const void* v, const bsa_mask* m,
                           void* out, float* lse, int BH, int n_valid, int n_pad, float scale,
                           cudaStream_t stream) {
-  using C = Cfg<D, BLK>;
+  using C = Cfg<D, BQ, BK>;
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(bsa_forward_kernel<D, BLK>,
+    if (cudaFuncSetAttribute(bsa_forward_kernel<D, BQ, BK>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(C::kSmemBytes)) != cudaSuccess)
       return BSA_ERR_LAUNCH;
@@ -580,7 +583,7 @@ bsa_status launch_forward(const void* q, const void* k, const void* v, const bsa
   }
   const int64_t rows = int64_t(BH) * n_pad;
   CUtensorMap tk, tv;
-  if (!make_map(&tk, k, rows, D, BLK) || !make_map(&tv, v, rows, D, BLK)) return BSA_ERR_LAUNCH;
+  if (!make_map(&tk, k, rows, D, BK) || !make_map(&tv, v, rows, D, BK)) return BSA_ERR_LAUNCH;
   FwdParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.bits = m->bits;
@@ -588,37 +591,41 @@ bsa_status launch_forward(const void* q, const void* k, const void* v, const bsa
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.BH = BH;
-  p.nb = n_pad / BLK;
-  p.words = (p.nb + 31) / 32;
+  p.nb_q = n_pad / BQ;
+  p.nb_k = n_pad / BK;
+  p.words = (p.nb_k + 31) / 32;
   p.n_valid = n_valid;
   p.n_pad = n_pad;
-  p.tiles_per_head = (p.nb + C::R - 1) / C::R;
-  p.num_tiles = C::R == 1 ? BH * p.nb : BH * p.tiles_per_head;
+  p.tiles_per_head = (p.nb_q + C::R - 1) / C::R;
+  p.num_tiles = C::R == 1 ? BH * p.nb_q : BH * p.tiles_per_head;
   p.scale_log2 = scale * 1.4426950408889634f;
   const int sms = bsa::num_sms();
   if (sms <= 0) return BSA_ERR_LAUNCH;
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-  bsa_forward_kernel<D, BLK><<<grid, kThreads, C::kSmemBytes, stream>>>(tk, tv, p);
+  bsa_forward_kernel<D, BQ, BK><<<grid, kThreads, C::kSmemBytes, stream>>>(tk, tv, p);
   return bsa::launch_status();
 }
 
 }  // namespace
 
-extern "C" bsa_status bsa_forward(const void* q, const void* k, const void* v,
-                                  const bsa_mask* mask, void* out, float* lse, int B, int H,
-                                  int n_valid, int n_pad, int d, int block, float softmax_scale,
-                                  void* stream) {
+extern "C" bsa_status bsa_forward_blocks(const void* q, const void* k, const void* v,
+                                         const bsa_mask* mask, void* out, float* lse, int B,
+                                         int H, int n_valid, int n_pad, int d, int block_q,
+                                         int block_k, float softmax_scale, void* stream) {
   if (!q || !k || !v || !mask || !out || !lse) return BSA_ERR_INVALID_ARG;
   if (!mask->bits || !mask->schedule) return BSA_ERR_INVALID_ARG;
-  if (B <= 0 || H <= 0 || n_pad <= 0 || n_valid <= 0 || block <= 0 || d <= 0)
+  if (B <= 0 || H <= 0 || n_pad <= 0 || n_valid <= 0 || block_q <= 0 || block_k <= 0 || d <= 0)
     return BSA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
-  if (block != 64 && block != 128) return BSA_ERR_UNSUPPORTED;
-  if (n_pad % block != 0) return BSA_ERR_UNSUPPORTED;
-  if (n_valid > n_pad || n_valid <= n_pad - block) return BSA_ERR_INVALID_ARG;
-  const int nb = n_pad / block;
-  if (mask->B != B || mask->H != H || mask->nb_q != nb || mask->nb_k != nb ||
-      mask->words != (nb + 31) / 32)
+  const bool same = block_q == block_k && (block_q == 64 || block_q == 128);
+  const bool finer_keys = block_q == 128 && block_k == 64;
+  if (!same && !finer_keys) return BSA_ERR_UNSUPPORTED;
+  if (n_pad % block_q != 0 || n_pad % block_k != 0) return BSA_ERR_UNSUPPORTED;
+  // only the last key block (and the last query block) may hold pad tokens
+  if (n_valid > n_pad || n_valid <= n_pad - block_k) return BSA_ERR_INVALID_ARG;
+  const int nb_q = n_pad / block_q, nb_k = n_pad / block_k;
+  if (mask->B != B || mask->H != H || mask->nb_q != nb_q || mask->nb_k != nb_k ||
+      mask->words != (nb_k + 31) / 32)
     return BSA_ERR_INVALID_ARG;
   if (int64_t(B) * H * n_pad >= (int64_t(1) << 31)) return BSA_ERR_OVERFLOW;
   if (!bsa::aligned16(q) || !bsa::aligned16(k) || !bsa::aligned16(v) || !bsa::aligned16(out) ||
@@ -627,13 +634,27 @@ extern "C" bsa_status bsa_forward(const void* q, const void* k, const void* v,
   const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf(float(d));
   const int BH = B * H;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 128 && block == 128)
-    return launch_forward<128, 128>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
-  if (d == 128 && block == 64)
-    return launch_forward<128, 64>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
-  if (d == 64 && block == 128)
-    return launch_forward<64, 128>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
-  return launch_forward<64, 64>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
+  if (d == 128) {
+    if (finer_keys)
+      return launch_forward<128, 128, 64>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
+    if (block_q == 128)
+      return launch_forward<128, 128, 128>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
+    return launch_forward<128, 64, 64>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
+  }
+  if (finer_keys)
+    return launch_forward<64, 128, 64>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
+  if (block_q == 128)
+    return launch_forward<64, 128, 128>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
+  return launch_forward<64, 64, 64>(q, k, v, mask, out, lse, BH, n_valid, n_pad, scale, s);
+}
+
+extern "C" bsa_status bsa_forward(const void* q, const void* k, const void* v,
+                                  const bsa_mask* mask, void* out, float* lse, int B, int H,
+                                  int n_valid, int n_pad, int d, int block, float softmax_scale,
+                                  void* stream) {
+  if (block != 64 && block != 128 && block > 0) return BSA_ERR_UNSUPPORTED;
+  return bsa_forward_blocks(q, k, v, mask, out, lse, B, H, n_valid, n_pad, d, block, block,
+                            softmax_scale, stream);
 }
 
 extern "C" bsa_status bsa_get_device_error(bsa_status* device_status) {

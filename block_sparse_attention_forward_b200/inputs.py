@@ -308,6 +308,27 @@ def gen_top_p_params(w: Workload, seed: int | None = None):
     return tau, top_p
 
 
+FINE_DROP = 0.3  # share of the 64-key halves of kept blocks that a finer mask drops
+
+
+def gen_mask_fine(w: Workload, q: torch.Tensor | None = None, k: torch.Tensor | None = None,
+                  seed: int | None = None) -> np.ndarray:
+    """Mask with key blocks of w.block // 2 tokens: [B, H, nb, 2 * nb].
+
+    The workload's own mask at w.block granularity, each kept key block split
+    into its two halves and each half dropped with probability FINE_DROP (a
+    finer mask keeps fewer unneeded keys: the granularity the pages name as the
+    bottleneck below 40 % density); both halves of the diagonal block stay."""
+    coarse = gen_mask(w, q, k, seed)
+    rng = np.random.default_rng((w.seed if seed is None else seed) + 6000)
+    fine = np.repeat(coarse, 2, axis=3)
+    fine[rng.random(fine.shape) < FINE_DROP] = 0
+    i = np.arange(w.nb)
+    fine[:, :, i, 2 * i] = 1
+    fine[:, :, i, 2 * i + 1] = 1
+    return fine
+
+
 def kept_tiles(mask: np.ndarray) -> int:
     return int(np.count_nonzero(mask))
 

@@ -320,6 +320,25 @@ bsa_status bsa_forward(const void* q, const void* k, const void* v, const bsa_ma
                        void* out, float* lse, int B, int H, int n_valid, int n_pad, int d,
                        int block, float softmax_scale, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * bsa_forward_blocks -- bsa_forward with query blocks of block_q tokens and
+ * key blocks of block_k tokens: query i and key j fall in blocks i / block_q
+ * and j / block_k, and the mask (from bsa_pack_mask on a dense
+ * [B, H, n_pad / block_q, n_pad / block_k] mask) has nb_q = n_pad / block_q
+ * rows of nb_k = n_pad / block_k bits.  block_q = 128 with block_k = 64 halves
+ * the key granularity: the 128 x 128 block is the granularity bottleneck the
+ * pages name below 40 % density (Sec. 5.4), and finer key blocks keep fewer
+ * unneeded keys per kept block.
+ *
+ * Supported (block_q, block_k): (128, 128), (64, 64), (128, 64); n_pad a
+ * multiple of both; n_pad - block_k < n_valid <= n_pad.  bsa_forward(...,
+ * block, ...) is bsa_forward_blocks(..., block, block, ...).  Arguments,
+ * outputs and errors otherwise as for bsa_forward.
+ * ------------------------------------------------------------------------- */
+bsa_status bsa_forward_blocks(const void* q, const void* k, const void* v, const bsa_mask* mask,
+                              void* out, float* lse, int B, int H, int n_valid, int n_pad, int d,
+                              int block_q, int block_k, float softmax_scale, void* stream);
+
 /* Reads and clears the device-side error word of the current device (set by a
  * kernel that timed out on a barrier).  Synchronises the current device.
  * Returns BSA_OK or BSA_ERR_TIMEOUT in *device_status; the return value is

@@ -21,8 +21,8 @@ def stratified_query_blocks(mask: np.ndarray, per_head: int, seed: int):
     """Query blocks to check per (b, h): the most-kept, the least-kept, the last
     (tail) block, block 0 and seeded random ones, as flat (bh, qb) pairs."""
     BH = mask.shape[0] * mask.shape[1]
-    nb = mask.shape[-1]
-    m = mask.reshape(BH, nb, nb)
+    nb = mask.shape[-2]  # query blocks (key blocks may be finer)
+    m = mask.reshape(BH, nb, mask.shape[-1])
     counts = m.sum(-1)
     rng = np.random.default_rng(seed)
     picks = []

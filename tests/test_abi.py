@@ -113,6 +113,24 @@ def test_host_orders_reject_bad_args(lib):
     assert lib.bsa_order_tables(buf, 8, 7, buf, buf) == 1  # n_pad < n
 
 
+def test_forward_blocks_rejects_bad_args(lib):
+    from block_sparse_attention_forward_b200._ffi import BsaMask
+    P = ctypes.c_void_p
+    a = P(0x10000)
+    fwd = lib.bsa_forward_blocks
+    # 128-row query blocks over 64-key blocks: nb_q = 8, nb_k = 16, 1 word
+    good = BsaMask(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 1, 2, 8, 16, 1)
+
+    def call(m=good, bq=128, bk=64, n_valid=1000, n_pad=1024, d=128):
+        return fwd(a, a, a, ctypes.byref(m), a, a, 1, 2, n_valid, n_pad, d, bq, bk, 0.0, None)
+    assert call(bq=64, bk=128) == 2                      # finer queries than keys
+    assert call(bq=128, bk=32) == 2
+    assert call(n_valid=960) == 1                        # pad fills a whole 64-key block
+    square = BsaMask(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 1, 2, 8, 8, 1)
+    assert call(m=square) == 1                           # mask built for 128-key blocks
+    assert call(d=96) == 2
+
+
 def test_permute_rejects_bad_args(lib):
     P = ctypes.c_void_p
     a, b = P(0x1000), P(0x2000)
