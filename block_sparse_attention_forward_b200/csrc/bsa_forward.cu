@@ -29,7 +29,12 @@
 //     key blocks its own query block did not keep.  Key blocks may be smaller
 //     than query blocks (128-row query blocks over 64-key blocks: twice the
 //     CRM bits per row, the finer key granularity Sec. 5.4 asks for below 40 %
-//     density); a kept key block is then an M = 128, N = 64 product.
+//     density).  Such blocks are taken in pairs of consecutive kept blocks:
+//     the producer loads the two 64-row K (and V) tiles into the two halves of
+//     one 128-row ring slot, so every product and softmax pass covers 128
+//     keys and the per-tile costs are paid once per pair; a lone last block
+//     is loaded into both halves (the second half is masked), so every value
+//     the tensor core reads is finite.
 //   * every barrier wait is bounded (about two seconds); a wait that runs out
 //     records BSA_ERR_TIMEOUT in a device word, the CTA drains what it has in
 //     flight and exits.
@@ -71,8 +76,10 @@ struct FwdParams {
 template <int D, int BQ, int BK>
 struct Cfg {
   static constexpr int R = kTileM / BQ;                         // query blocks per tile
+  static constexpr bool kPairs = BQ == 128 && BK == 64;         // two key blocks per S tile
+  static constexpr int kTileN = kPairs ? 2 * BK : BK;           // keys per S tile and ring slot
   static constexpr int kRegions = D / 64;                       // 128-byte column groups
-  static constexpr uint32_t kKVRegion = BK * 128;
+  static constexpr uint32_t kKVRegion = kTileN * 128;
   static constexpr uint32_t kSlotBytes = kRegions * kKVRegion;  // one K or V tile
   static constexpr uint32_t kMaxSmem = 227u * 1024u;
   static constexpr int kFitStages = int((kMaxSmem - 256 - 1024) / kSlotBytes);
@@ -83,7 +90,7 @@ struct Cfg {
   // fits on the SM (each CTA owns all 512 TMEM columns)
   static constexpr uint32_t kSmemUsed = kOffBar + 256 + 1024;
   static constexpr uint32_t kSmemBytes = kSmemUsed > 120u * 1024u ? kSmemUsed : 120u * 1024u;
-  static constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, BK, false);
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false);
   static_assert(kSmemUsed <= kMaxSmem, "shared memory budget");
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, true);
 };
@@ -236,8 +243,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (union_count(t, p.words) == 0) continue;
         CrmIter it;
         it.init(t.row0, t.row1, p.words);
-        for (int j = it.index(); j >= 0; it.next(), j = it.index()) {
+        for (int j = it.index(); j >= 0;) {
+          int j2 = -1;  // second key block of the pair (pairs only)
+          if constexpr (C::kPairs) {
+            it.next();
+            j2 = it.index();
+          }
           const int32_t kv_row = t.bh * p.n_pad + j * BK;
+          const int32_t kv_row2 = t.bh * p.n_pad + (j2 >= 0 ? j2 : j) * BK;
 #pragma unroll
           for (int kv = 0; kv < 2; ++kv) {  // K then V
             const uint32_t slot = item % C::kStages;
@@ -251,11 +264,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(fbar, C::kSlotBytes);
             const uint32_t dst = sKV + slot * C::kSlotBytes;
 #pragma unroll
-            for (int r = 0; r < C::kRegions; ++r)
+            for (int r = 0; r < C::kRegions; ++r) {
               tma_load_2d(dst + r * C::kKVRegion, kv == 0 ? &tm_k : &tm_v, fbar, r * 64, kv_row);
+              if constexpr (C::kPairs)  // rows BK.. of the slot: the pair's second block
+                tma_load_2d(dst + r * C::kKVRegion + BK * 128, kv == 0 ? &tm_k : &tm_v, fbar,
+                            r * 64, kv_row2);
+            }
             ++item;
           }
           if (!ok) break;
+          if (!C::kPairs || j2 >= 0) it.next();
+          j = it.index();
         }
       }
       if (!ok) {
@@ -283,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // keys (2048 bytes) per step
         const uint32_t v_base = sKV + slot * C::kSlotBytes;
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
+        for (int kk = 0; kk < C::kTileN / 16; ++kk) {
           const uint64_t bdesc = smem_desc_sw128(v_base + kk * 16 * 128, C::kKVRegion, 1024);
           mma_ts(tmem + kTmemO, p_tmem + kk * 8, bdesc, C::kIdescPV, (first && kk == 0) ? 0u : 1u);
         }
@@ -293,8 +312,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         const TileInfo t = tile_info<C::R>(p, tile);
-        const int cnt = union_count(t, p.words);
-        if (cnt == 0) continue;
+        const int kept = union_count(t, p.words);
+        if (kept == 0) continue;
+        const int cnt = C::kPairs ? (kept + 1) / 2 : kept;  // S tiles of this query tile
         if (!wait_barrier(smem_addr(&bars->q_full), q_iter & 1, abort)) {
           ok = false;
           break;
@@ -382,7 +402,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       CrmIter it;
       it.init(t.row0, t.row1, p.words);
       int n = 0;
-      for (int j = it.index(); j >= 0; it.next(), j = it.index(), ++n) {
+      for (int j = it.index(); j >= 0; ++n) {
+        int j2 = -1;  // second key block of the pair (pairs only)
+        if constexpr (C::kPairs) {
+          it.next();
+          j2 = it.index();
+        }
         const uint32_t gi = g + n, sb = gi & 1;
         // tcgen05.ld/st below are warp-collective: agree on the outcome first
         if (!__all_sync(0xffffffffu, wait_barrier(smem_addr(&bars->s_full[sb]), (gi >> 1) & 1,
@@ -392,12 +417,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t s_tmem = tmem + lane_base + (sb ? kTmemS1 : kTmemS0);
-        uint32_t sr[BK];  // raw fp32 scores of this row, one tcgen05.ld
-        if constexpr (BK == 128) tmem_load128(s_tmem, sr);
+        uint32_t sr[C::kTileN];  // raw fp32 scores of this row, one tcgen05.ld
+        if constexpr (C::kTileN == 128) tmem_load128(s_tmem, sr);
         else tmem_load64(s_tmem, sr);
         bool member = row_in_head;
         if (C::R > 1 && member) member = (__ldg(my_bits + (j >> 5)) >> (j & 31)) & 1u;
-        if (has_tail && j == p.nb_k - 1) {
+        if constexpr (C::kPairs) {
+          if (j2 < 0) {  // a lone block: its copy in the second half does not count
+#pragma unroll
+            for (int c = BK; c < 2 * BK; ++c) sr[c] = __float_as_uint(-INFINITY);
+          }
+          // the last key block, in whichever half it sits (static indices keep
+          // sr in registers)
+          const int valid = p.n_valid - (p.nb_k - 1) * BK;
+          if (has_tail && j == p.nb_k - 1) {
+#pragma unroll
+            for (int c = 0; c < BK; ++c)
+              if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+          }
+          if (has_tail && j2 == p.nb_k - 1) {
+#pragma unroll
+            for (int c = 0; c < BK; ++c)
+              if (c >= valid) sr[BK + c] = __float_as_uint(-INFINITY);
+          }
+        } else if (has_tail && j == p.nb_k - 1) {
           const int valid = p.n_valid - j * BK;
 #pragma unroll
           for (int c = 0; c < BK; ++c)
@@ -407,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(sr[i]);
 #pragma unroll
-        for (int c = 8; c < BK; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+        for (int c = 8; c < C::kTileN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         // Lazy rescale: the reference max only moves when the row max grows by
@@ -450,9 +493,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) sum8[i] = 0.0f;
         const float neg_m = -m_new;
-        uint32_t pk[BK / 2];
+        uint32_t pk[C::kTileN / 2];
 #pragma unroll
-        for (int i = 0; i < BK / 2; ++i) {
+        for (int i = 0; i < C::kTileN / 2; ++i) {
           float p0 = 0.0f, p1 = 0.0f;
           if (member) {
             p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), p.scale_log2, neg_m));
@@ -464,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // P overwrites the first half of this S buffer: packed bf16 pairs, one
         // 32-bit column per two keys
-        if constexpr (BK == 128) tmem_store64(s_tmem, pk);
+        if constexpr (C::kTileN == 128) tmem_store64(s_tmem, pk);
         else tmem_store32(s_tmem, pk);
         const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
                           ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
@@ -475,6 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_store_wait();
         tc_fence_before();
         mbar_arrive(smem_addr(&bars->p_full[sb]));
+        if (!C::kPairs || j2 >= 0) it.next();
+        j = it.index();
       }
       if (!ok) break;
 
