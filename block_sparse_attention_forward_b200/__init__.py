@@ -28,7 +28,8 @@ from ._ffi import BsaError, BsaMask
 
 __all__ = ["BsaError", "PackedMask", "pack_mask", "pack_mask_from_threshold",
            "threshold_resize", "predict_top_p", "tile_permute", "tile_unpermute", "hilbert_order", "tile_order",
-           "order_tables", "gather_rows", "forward", "device_error", "version"]
+           "order_tables", "gather_rows", "forward", "attention_host", "device_error",
+           "version"]
 
 
 def _stream(device: torch.device) -> ctypes.c_void_p:
@@ -297,6 +298,45 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask: PackedMask,
                                     int(block), int(block_k), float(softmax_scale or 0.0),
                                     _stream(q.device))
         _ffi.check(st, "bsa_forward_blocks")
+    return out, lse
+
+
+def attention_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask: torch.Tensor, grid,
+                   tile, block: int, softmax_scale: float | None = None,
+                   heads_per_chunk: int = 0, out: torch.Tensor | None = None,
+                   lse: torch.Tensor | None = None, device: torch.device | None = None):
+    """The whole path from host tensors to host tensors on the current (or given)
+    GPU, copies overlapped with the kernels (bsa_attention_host).
+
+    q, k, v: host bf16 [B, H, T*Hs*Ws, d] frame-major (pinned for overlap);
+    mask: host uint8 [B, H, nb, nb].  Returns (out host bf16 [B, H, N, d]
+    frame-major, lse host fp32 [B, H, n_pad] tile-major); both are complete once
+    the current stream has finished."""
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host bf16 tensor")
+    if mask.is_cuda or mask.dtype != torch.uint8 or not mask.is_contiguous():
+        raise ValueError("mask must be a contiguous host uint8 tensor")
+    B, H, N, d = q.shape
+    T, Hs, Ws, tt, th, tw = _grid_args(grid, tile)
+    if N != T * Hs * Ws or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must be [B, H, T*Hs*Ws, d]")
+    n_pad = -(-N // block) * block
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if out is None:
+        out = torch.empty_like(q, pin_memory=q.is_pinned())
+    if lse is None:
+        lse = torch.empty((B, H, n_pad), dtype=torch.float32, pin_memory=q.is_pinned())
+    lib = _ffi.load()
+    ws_bytes = lib.bsa_attention_host_workspace(B, H, T, Hs, Ws, d, int(block), int(heads_per_chunk))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    st = lib.bsa_attention_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), mask.data_ptr(),
+                                out.data_ptr(), lse.data_ptr(), B, H, T, Hs, Ws, d, tt, th, tw,
+                                int(block), float(softmax_scale or 0.0), int(heads_per_chunk),
+                                ws.data_ptr(), ws.numel(), _stream(dev))
+    _ffi.check(st, "bsa_attention_host")
+    # the workspace must outlive the queued work: keep it until the stream drains
+    ws.record_stream(torch.cuda.current_stream(dev))
     return out, lse
 
 

@@ -41,6 +41,8 @@ EXPORTED = (
     "bsa_tile_unpermute",
     "bsa_forward",
     "bsa_forward_blocks",
+    "bsa_attention_host_workspace",
+    "bsa_attention_host",
     "bsa_get_device_error",
 )
 
@@ -115,6 +117,11 @@ def load() -> ctypes.CDLL:
     lib.bsa_forward_blocks.argtypes = [P, P, P, ctypes.POINTER(BsaMask), P, P, I, I, I, I, I, I,
                                        I, ctypes.c_float, P]
     lib.bsa_forward_blocks.restype = I
+    lib.bsa_attention_host_workspace.argtypes = [I, I, I, I, I, I, I, I]
+    lib.bsa_attention_host_workspace.restype = SZ
+    lib.bsa_attention_host.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I,
+                                       ctypes.c_float, I, P, SZ, P]
+    lib.bsa_attention_host.restype = I
     lib.bsa_get_device_error.argtypes = [ctypes.POINTER(I)]
     lib.bsa_get_device_error.restype = I
     _lib = lib

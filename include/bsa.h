@@ -339,6 +339,46 @@ bsa_status bsa_forward_blocks(const void* q, const void* k, const void* v, const
                               void* out, float* lse, int B, int H, int n_valid, int n_pad, int d,
                               int block_q, int block_k, float softmax_scale, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * bsa_attention_host -- the whole path from HOST buffers to HOST buffers:
+ * bsa_pack_mask, bsa_tile_permute of q, k, v, bsa_forward and
+ * bsa_tile_unpermute, with the host <-> device copies overlapped with the
+ * kernels.
+ *
+ * Heads are independent (each has its own mask, token order and softmax), so
+ * the B*H heads run in chunks of heads_per_chunk (<= 0: about B*H / 8) as a
+ * three-stage pipeline: chunk c + 1 is copied in and chunk c - 1 copied out
+ * while chunk c computes on `stream`.  Two auxiliary streams per device (made
+ * on first use) carry the copies; they start after the work already queued on
+ * `stream` and are joined back into it, so the call is ordered on `stream`
+ * like any other.  Calls on one device from several host threads at once
+ * share those streams and run one after the other.
+ *
+ *   q, k, v  HOST [B, H, N, d] bf16, frame-major (N = T*Hs*Ws).  Pinned
+ *            (page-locked) memory lets the copies overlap; pageable memory
+ *            works but copies synchronously.
+ *   mask     HOST [B, H, nb, nb] uint8, nb = n_pad / block,
+ *            n_pad = ceil(N / block) * block.
+ *   out      HOST [B, H, N, d] bf16, frame-major (as bsa_tile_unpermute).
+ *   lse      HOST [B, H, n_pad] fp32 in tile-major order (as bsa_forward).
+ *   tt, th, tw, block, softmax_scale: as for bsa_tile_permute / bsa_forward.
+ *   workspace  DEVICE scratch of bsa_attention_host_workspace(...) bytes,
+ *            256-byte aligned (two chunks' buffers).
+ *
+ * The host buffers must stay valid until the work on `stream` completes.
+ * Errors: BSA_ERR_INVALID_ARG, BSA_ERR_OVERFLOW, BSA_ERR_WORKSPACE,
+ * BSA_ERR_MISALIGNED, BSA_ERR_LAUNCH, and any error of the calls above (for
+ * example BSA_ERR_UNSUPPORTED for d = 96).  After an error part of the
+ * pipeline may already be queued.
+ * ------------------------------------------------------------------------- */
+size_t bsa_attention_host_workspace(int B, int H, int T, int Hs, int Ws, int d, int block,
+                                    int heads_per_chunk);
+bsa_status bsa_attention_host(const void* q, const void* k, const void* v, const uint8_t* mask,
+                              void* out, float* lse, int B, int H, int T, int Hs, int Ws, int d,
+                              int tt, int th, int tw, int block, float softmax_scale,
+                              int heads_per_chunk, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
 /* Reads and clears the device-side error word of the current device (set by a
  * kernel that timed out on a barrier).  Synchronises the current device.
  * Returns BSA_OK or BSA_ERR_TIMEOUT in *device_status; the return value is

@@ -131,6 +131,23 @@ def test_forward_blocks_rejects_bad_args(lib):
     assert call(d=96) == 2
 
 
+def test_attention_host_rejects_bad_args(lib):
+    P = ctypes.c_void_p
+    a = P(0x10000)
+    ws = P(0x100000)
+    fn = lib.bsa_attention_host
+    need = lib.bsa_attention_host_workspace(1, 2, 4, 16, 16, 64, 64, 0)
+    assert need > 0
+
+    def call(q=a, ws_ptr=ws, ws_bytes=need, d=64, block=64):
+        return fn(q, a, a, a, a, a, 1, 2, 4, 16, 16, d, 1, 8, 8, block, 0.0, 0, ws_ptr, ws_bytes,
+                  None)
+    assert call(q=None) == 1
+    assert call(ws_ptr=None) == 1
+    assert call(ws_bytes=need - 1) == 7
+    assert call(ws_ptr=P(0x100010)) == 3  # 256-byte alignment
+
+
 def test_permute_rejects_bad_args(lib):
     P = ctypes.c_void_p
     a, b = P(0x1000), P(0x2000)
