@@ -346,7 +346,7 @@ bsa_status bsa_forward_blocks(const void* q, const void* k, const void* v, const
  * kernels.
  *
  * Heads are independent (each has its own mask, token order and softmax), so
- * the B*H heads run in chunks of heads_per_chunk (<= 0: about B*H / 8) as a
+ * the B*H heads run in chunks of heads_per_chunk (<= 0: ceil(B*H / 16)) as a
  * three-stage pipeline: chunk c + 1 is copied in and chunk c - 1 copied out
  * while chunk c computes on `stream`.  Two auxiliary streams per device (made
  * on first use) carry the copies; they start after the work already queued on
