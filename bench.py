@@ -559,7 +559,7 @@ def main():
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     next_rows = None
-    if not args.no_next:
+    if not args.no_next and world == 1:  # extra rows only at N = 1: no GPU held longer
         next_rows = measure_threshold_rows(w, dev, stream, float(peaks["hbm_gbs"]))
         next_rows.update(measure_order_rows(w, dev, stream, float(peaks["hbm_gbs"])))
         next_rows.update(measure_predict_row(w, dev, stream, float(peaks["hbm_gbs"])))
