@@ -618,14 +618,12 @@ bsa_status launch_forward(const void* q, const void* k, const void* v, const bsa
                           void* out, float* lse, int BH, int n_valid, int n_pad, float scale,
                           cudaStream_t stream) {
   using C = Cfg<D, BQ, BK>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(bsa_forward_kernel<D, BQ, BK>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(C::kSmemBytes)) != cudaSuccess)
-      return BSA_ERR_LAUNCH;
-    attr_set = true;
-  }
+  // set on every call: the attribute belongs to the current device, and one
+  // process may launch on several
+  if (cudaFuncSetAttribute(bsa_forward_kernel<D, BQ, BK>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(C::kSmemBytes)) != cudaSuccess)
+    return BSA_ERR_LAUNCH;
   const int64_t rows = int64_t(BH) * n_pad;
   CUtensorMap tk, tv;
   if (!make_map(&tk, k, rows, D, BK) || !make_map(&tv, v, rows, D, BK)) return BSA_ERR_LAUNCH;
