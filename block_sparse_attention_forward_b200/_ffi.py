@@ -43,6 +43,7 @@ EXPORTED = (
     "bsa_forward_blocks",
     "bsa_attention_host_workspace",
     "bsa_attention_host",
+    "bsa_check_wait_timeout",
     "bsa_get_device_error",
 )
 
@@ -122,6 +123,8 @@ def load() -> ctypes.CDLL:
     lib.bsa_attention_host.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I,
                                        ctypes.c_float, I, P, SZ, P]
     lib.bsa_attention_host.restype = I
+    lib.bsa_check_wait_timeout.argtypes = [ctypes.c_uint, P]
+    lib.bsa_check_wait_timeout.restype = I
     lib.bsa_get_device_error.argtypes = [ctypes.POINTER(I)]
     lib.bsa_get_device_error.restype = I
     _lib = lib

@@ -107,13 +107,14 @@ struct Barriers {
 
 // Bounded wait, slow path: spin until the phase of `parity` completed (true)
 // or this CTA gives up (timeout here, or another role already aborted).
-__device__ __noinline__ bool wait_barrier_slow(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ __noinline__ bool wait_barrier_slow(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               uint64_t timeout_ns = kTimeoutNs) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kTimeoutNs) {
+      if (global_timer_ns() - t0 > timeout_ns) {
         *abort = 1;
         atomicExch(&g_bsa_device_error, int(BSA_ERR_TIMEOUT));
         return false;
@@ -578,6 +579,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Failure-path check: one thread waits on an mbarrier that nothing arrives on,
+// through the same bounded wait the forward uses; it gives up after
+// timeout_ns, records BSA_ERR_TIMEOUT and returns.
+__global__ void wait_timeout_check_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&bar), 1);
+    abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_barrier_slow(smem_addr(&bar), 0, &abort, timeout_ns);
+}
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -698,6 +714,13 @@ extern "C" bsa_status bsa_forward(const void* q, const void* k, const void* v,
   if (block != 64 && block != 128 && block > 0) return BSA_ERR_UNSUPPORTED;
   return bsa_forward_blocks(q, k, v, mask, out, lse, B, H, n_valid, n_pad, d, block, block,
                             softmax_scale, stream);
+}
+
+extern "C" bsa_status bsa_check_wait_timeout(unsigned timeout_us, void* stream) {
+  if (timeout_us == 0 || timeout_us > 10000000u) return BSA_ERR_INVALID_ARG;
+  wait_timeout_check_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      uint64_t(timeout_us) * 1000ull);
+  return bsa::launch_status();
 }
 
 extern "C" bsa_status bsa_get_device_error(bsa_status* device_status) {

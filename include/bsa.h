@@ -379,6 +379,14 @@ bsa_status bsa_attention_host(const void* q, const void* k, const void* v, const
                               int heads_per_chunk, void* workspace, size_t workspace_bytes,
                               void* stream);
 
+/* Failure-path check (no counterpart in the paper): launches one thread that
+ * waits on a pipeline barrier nothing will complete, through the same bounded
+ * wait the forward kernel uses, so that the wait runs out after timeout_us
+ * microseconds (1 .. 10^7) and records BSA_ERR_TIMEOUT for
+ * bsa_get_device_error.  Nothing faults, traps or hangs: the kernel returns
+ * and the context stays usable.  Errors: BSA_ERR_INVALID_ARG, BSA_ERR_LAUNCH. */
+bsa_status bsa_check_wait_timeout(unsigned timeout_us, void* stream);
+
 /* Reads and clears the device-side error word of the current device (set by a
  * kernel that timed out on a barrier).  Synchronises the current device.
  * Returns BSA_OK or BSA_ERR_TIMEOUT in *device_status; the return value is

@@ -148,6 +148,11 @@ def test_attention_host_rejects_bad_args(lib):
     assert call(ws_ptr=P(0x100010)) == 3  # 256-byte alignment
 
 
+def test_wait_timeout_check_rejects_bad_args(lib):
+    assert lib.bsa_check_wait_timeout(0, None) == 1
+    assert lib.bsa_check_wait_timeout(10000001, None) == 1
+
+
 def test_permute_rejects_bad_args(lib):
     P = ctypes.c_void_p
     a, b = P(0x1000), P(0x2000)
