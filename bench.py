@@ -20,8 +20,10 @@ After the timed steps, `next_rows` reports further steps measured on their own
 (L2 flushed before each call): bsa_pack_mask_from_threshold at the workload's
 block grid, bsa_threshold_resize of a 480p-grid map to it, bsa_gather_rows
 applying the Hilbert-curve order and head-aware tile orders to one tensor,
-the online top-p predictor bsa_predict_top_p on the workload's q and k, and the
-forward with 64-token key blocks under 128-token query blocks.
+the online top-p predictor bsa_predict_top_p on the workload's q and k, the
+forward with 64-token key blocks under 128-token query blocks, and the forward
+on an all-ones mask (the speedup of the workload's mask over it; PyTorch's dense
+SDPA on the same tensors as context).
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of query blocks of the same workload (rank 0 only).
@@ -171,9 +173,12 @@ def _bits(x: torch.Tensor) -> np.ndarray:
     return x.contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def oracle_sample(w, q, k, v, mask, budget_s: float, seed: int):
+def oracle_sample(w, q, k, v, mask, budget_s: float, seed: int, gpu_out=None, gpu_lse=None):
     """Times the oracle on whole query blocks (all rows) of the workload until
-    about budget_s of CPU work; returns (tflops_equivalent, seconds, blocks, cores)."""
+    about budget_s of CPU work; returns (tflops_equivalent, seconds, blocks, cores,
+    errors).  With the GPU's tile-major output and LSE ([B, H, n_pad, d] and
+    [B, H, n_pad] on the host) the same rows are compared: errors = (max abs,
+    mean abs, LSE max abs, rows), else None."""
     import oracle
     BH = w.B * w.H
     perm = oracle.tile_order(w.T, w.Hs, w.Ws, w.tt, w.th, w.tw)
@@ -188,18 +193,32 @@ def oracle_sample(w, q, k, v, mask, budget_s: float, seed: int):
     flops = 0.0
     spent = 0.0
     blocks = 0
+    err_max = err_sum = lse_max = 0.0
+    err_n = 0
     order = [(int(bh), int(qb)) for qb in rng.permutation(w.nb) for bh in heads]
     for bh, qb in order:
         qp, kp, vp = per_head[bh]
         rows = (qb * w.block + np.arange(w.block)).astype(np.int64)
         t0 = time.perf_counter()
-        oracle.attention(qp, kp, vp, m[bh:bh + 1], w.n, w.block, rows=rows)
+        ref, ref_lse = oracle.attention(qp, kp, vp, m[bh:bh + 1], w.n, w.block, rows=rows)
         spent += time.perf_counter() - t0
         flops += 4.0 * w.d * w.block * w.block * float(m[bh, qb].sum())
         blocks += 1
+        if gpu_out is not None:
+            got = gpu_out.reshape(BH, w.n_pad, w.d)[bh, rows].astype(np.float64)
+            diff = np.abs(got - ref)
+            err_max = max(err_max, float(diff.max()))
+            err_sum += float(diff.sum())
+            err_n += diff.size
+            gl = gpu_lse.reshape(BH, w.n_pad)[bh, rows].astype(np.float64)
+            fin = np.isfinite(ref_lse)
+            if fin.any():
+                lse_max = max(lse_max, float(np.abs(gl[fin] - ref_lse[fin]).max()))
         if spent >= budget_s:
             break
-    return flops / spent / 1e12, spent, blocks, oracle.num_threads()
+    errors = ((err_max, err_sum / max(err_n, 1), lse_max, blocks * w.block)
+              if gpu_out is not None else None)
+    return flops / spent / 1e12, spent, blocks, oracle.num_threads(), errors
 
 
 def run_reference(args, w):
@@ -212,7 +231,7 @@ def run_reference(args, w):
     per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     vals = []
     for i in range(args.warmup + args.steps):
-        tf, spent, blocks, cores = oracle_sample(w, q, k, v, mask, per_step, seed=w.seed + i)
+        tf, spent, blocks, cores, _ = oracle_sample(w, q, k, v, mask, per_step, seed=w.seed + i)
         if i >= args.warmup:
             vals.append((tf, spent, blocks))
     value = statistics.median([x[0] for x in vals])
@@ -387,6 +406,61 @@ def measure_finer_keys_row(w, dev, stream, peak_tflops: float):
                                    "frac": tf / peak_tflops, "bound": "tensor", "launches": 1}}
 
 
+def measure_dense_rows(w, dev, stream, peak_tflops: float, sparse_fwd_ms: float | None):
+    """The same forward on an all-ones mask (every tile kept) on the workload's
+    shapes, the speedup of the workload's mask over it (the pages compare their
+    kernel with dense FlashAttention the same way), and PyTorch's dense
+    scaled_dot_product_attention on the same tensors as context only."""
+    import block_sparse_attention_forward_b200 as bsa
+    q, k, v = I.gen_qkv(w, seed=w.seed + 8000)
+    grid, tile = (w.T, w.Hs, w.Ws), (w.tt, w.th, w.tw)
+    qp, kp, vp = (bsa.tile_permute(t.to(dev), grid, tile, w.n_pad) for t in (q, k, v))
+    del q, k, v
+    ones = torch.ones((w.B, w.H, w.nb, w.nb), dtype=torch.uint8, device=dev)
+    pm = bsa.pack_mask(ones)
+    out = torch.empty_like(qp)
+    lse = torch.empty((w.B, w.H, w.n_pad), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    us = time_device_us(lambda: bsa.forward(qp, kp, vp, pm, w.n, w.block, out=out, lse=lse),
+                        stream, flush, iters=3, warmup=2)
+    if bsa.device_error() != 0:
+        raise RuntimeError("device error in the dense forward")
+    flops = 4.0 * w.d * w.block * w.block * w.B * w.H * w.nb * w.nb
+    tf = flops / (us * 1e-6) / 1e12
+    res = {"forward_all_ones": {"us": us, "achieved_tflops": tf, "peak": peak_tflops,
+                                "frac": tf / peak_tflops, "bound": "tensor",
+                                "speedup_of_mask": (us * 1e-3 / sparse_fwd_ms)
+                                if sparse_fwd_ms else None}}
+    # time against density on the same shapes (Bernoulli masks, diagonal kept):
+    # the pages expect time to fall in proportion to the kept blocks
+    rng = np.random.default_rng(w.seed + 9000)
+    sweep = []
+    for dens in (0.5, 0.25, 0.10, 0.05):
+        m = (rng.random((w.B, w.H, w.nb, w.nb)) < dens).astype(np.uint8)
+        idx = np.arange(w.nb)
+        m[:, :, idx, idx] = 1
+        pm_d = bsa.pack_mask(torch.from_numpy(m).to(dev))
+        us_d = time_device_us(lambda: bsa.forward(qp, kp, vp, pm_d, w.n, w.block, out=out,
+                                                  lse=lse), stream, flush, iters=3, warmup=2)
+        kept = float(m.mean())
+        sweep.append({"density": kept, "us": us_d, "speedup_vs_all_ones": us / us_d,
+                      "time_over_density_x_all_ones": us_d / (kept * us),
+                      "achieved_tflops": flops * kept / (us_d * 1e-6) / 1e12})
+    res["density_sweep"] = sweep
+    # context only: dense attention over the N valid tokens with PyTorch's SDPA
+    qd, kd, vd = (t[:, :, :w.n] for t in (qp, kp, vp))
+    try:
+        sdpa = torch.nn.functional.scaled_dot_product_attention
+        us_t = time_device_us(lambda: sdpa(qd, kd, vd), stream, flush, iters=3, warmup=2)
+        tf_t = 4.0 * w.d * w.n * w.n * w.B * w.H / (us_t * 1e-6) / 1e12
+        res["torch_sdpa_dense_context"] = {"us": us_t, "achieved_tflops": tf_t,
+                                           "note": "context only, not ours"}
+    except RuntimeError as e:  # e.g. no fused kernel for the shape
+        res["torch_sdpa_dense_context"] = {"unavailable": str(e)[:120]}
+    del flush, qp, kp, vp, out
+    return res
+
+
 def workload_config(w, mask):
     kept = I.kept_tiles(mask)
     total = w.B * w.H * w.nb * w.nb
@@ -434,9 +508,9 @@ def main():
                                        float(peaks["hbm_gbs"])))
         rows.update(measure_predict_row(w, dev, torch.cuda.current_stream(dev),
                                         float(peaks["hbm_gbs"])))
-        rows.update(measure_finer_keys_row(w, dev, torch.cuda.current_stream(dev),
-                                           float(peaks.get("bf16_tflops_sustained",
-                                                           peaks.get("bf16_tflops")))))
+        pk = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        rows.update(measure_finer_keys_row(w, dev, torch.cuda.current_stream(dev), pk))
+        rows.update(measure_dense_rows(w, dev, torch.cuda.current_stream(dev), pk, None))
         if rank == 0:
             print(json.dumps({"workload": w.name, "next_rows": rows}), flush=True)
         if world > 1:
@@ -564,6 +638,7 @@ def main():
         next_rows.update(measure_order_rows(w, dev, stream, float(peaks["hbm_gbs"])))
         next_rows.update(measure_predict_row(w, dev, stream, float(peaks["hbm_gbs"])))
         next_rows.update(measure_finer_keys_row(w, dev, stream, peak))
+        next_rows.update(measure_dense_rows(w, dev, stream, peak, fwd_ms))
     fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
                 "frac": fwd_tflops / peak, "traffic": recorded_traffic(w.name),
@@ -572,11 +647,20 @@ def main():
                 "fwd_ms": fwd_ms}
 
     cpu = None
+    parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tf, spent, blocks, cores = oracle_sample(w, q, k, v, mask, 15.0, seed=w.seed)
+        # the last timed step's tile-major output and LSE, compared on the sampled rows
+        gpu_out = out_p.float().cpu().numpy()
+        gpu_lse = lse.cpu().numpy()
+        tf, spent, blocks, cores, errs = oracle_sample(w, q, k, v, mask, 15.0, seed=w.seed,
+                                                       gpu_out=gpu_out, gpu_lse=gpu_lse)
         cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{blocks} whole query blocks ({w.block} rows each) of 4 seeded heads, "
                          f"{spent:.1f} s of fp64 OpenMP oracle"}
+        parity = {"rows": errs[3], "out_max_abs": errs[0], "out_mean_abs": errs[1],
+                  "lse_max_abs": errs[2],
+                  "tolerance": {"out_max_abs": 2e-2, "out_mean_abs": 2e-3, "lse_max_abs": 1e-3},
+                  "against": "fp64 oracle on the cpu_baseline sample, last timed step's output"}
 
     if world > 1:
         torch.distributed.barrier()
@@ -590,6 +674,7 @@ def main():
             "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary(t_wall0, t_wall1),
             "peak_frac_step": value / peak,
+            "parity": parity,
             "next_rows": next_rows,
         }
         print(json.dumps(line), flush=True)
