@@ -28,7 +28,8 @@
 //     written by the softmax threads once per tile).  S(n+1) is computed
 //     while the softmax works on S(n).
 //   * work order: query tiles are taken from the count-descending schedule
-//     (heaviest first), CTA c handles tiles c, c + grid, ...
+//     (heaviest first) in rounds of one tile per CTA, alternating direction
+//     (snake_tile)
 //   * a tile is always 128 query rows; with 64-token query blocks it holds two
 //     query blocks and walks the union of their CRM rows, each row masking the
 //     key blocks its own query block did not keep.  Key blocks may be smaller
@@ -179,6 +180,16 @@ struct CrmIter {
   __device__ __forceinline__ int index() const { return val == 0u ? -1 : base + __ffs(val) - 1; }
 };
 
+// Tile of round r for this CTA.  Tiles come in schedule order (most kept
+// blocks first); rounds alternate direction (CTA b takes the b-th tile of an
+// even round and the b-th from the end of an odd one), so the heavy and light
+// ends of consecutive rounds pair up.  On the 720p workload the busiest CTA
+// then carries 0.25 % more than the mean, against 0.54 % with a plain stride.
+__device__ __forceinline__ int snake_tile(int r) {
+  const int G = int(gridDim.x), b = int(blockIdx.x);
+  return r * G + ((r & 1) ? G - 1 - b : b);
+}
+
 struct TileInfo {
   int bh, qb0;
   const uint32_t* row0;
@@ -256,7 +267,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t item = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+      for (int r = 0; r * int(gridDim.x) < p.num_tiles && ok; ++r) {
+        const int tile = snake_tile(r);
+        if (tile >= p.num_tiles) continue;
         const TileInfo t = tile_info<C::R>(p, tile);
         if (union_count(t, p.words) == 0) continue;
         CrmIter it;
@@ -344,7 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         return wait_fast(smem_addr(&bars->kv_full[it % C::kStages]), (it / C::kStages) & 1,
                             abort);
       };
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+      for (int r = 0; r * int(gridDim.x) < p.num_tiles && ok; ++r) {
+        const int tile = snake_tile(r);
+        if (tile >= p.num_tiles) continue;
         const TileInfo t = tile_info<C::R>(p, tile);
         const int kept = union_count(t, p.words);
         if (kept == 0) continue;
@@ -394,7 +409,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t g = 0;
     bool ok = true;
     const bool has_tail = p.n_valid < p.n_pad;
-    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+    for (int r = 0; r * int(gridDim.x) < p.num_tiles && ok; ++r) {
+      const int tile = snake_tile(r);
+      if (tile >= p.num_tiles) continue;
       const TileInfo t = tile_info<C::R>(p, tile);
       const int my_qb = t.qb0 + row / BQ;
       const bool row_in_head = my_qb < p.nb_q;
