@@ -23,13 +23,15 @@ inline int num_sms() {
   return sms;
 }
 
-// Stages 2-5 of mask packing (tiled count sort -> row_offsets and schedule,
-// then the kept-block lists), for any producer that has written every row's
+// Stages 2-7 of mask packing (tiled count sort -> row_offsets and schedule,
+// the head-mix check of that schedule and, when it mixes many heads, the
+// head-major order; then the kept-block lists), for any producer that has
+// written every row's
 // CRM words and count.  `scratch` holds pack_scratch_bytes(rows, nb_k) bytes,
 // 16-byte aligned.  Defined in bsa_pack.cu.
 size_t pack_scratch_bytes(int64_t rows, int nb_k);
-bsa_status pack_finish(const uint32_t* bits, const int32_t* counts, int rows, int nb_k,
-                       int32_t* row_offsets, int32_t* col_idx, int32_t* schedule,
+bsa_status pack_finish(const uint32_t* bits, const int32_t* counts, int rows, int nb_q,
+                       int nb_k, int32_t* row_offsets, int32_t* col_idx, int32_t* schedule,
                        void* scratch, cudaStream_t s);
 // Largest nb_k the packing stages accept (BSA_ERR_UNSUPPORTED beyond).
 constexpr int kPackMaxNbK = 49151;

@@ -227,9 +227,11 @@ __global__ void __launch_bounds__(kTileRows)
 // row_offsets[rows]); histograms -> first schedule slot of every (count, tile).
 __global__ void __launch_bounds__(kTileRows, 1)
     tile_scan_kernel(int rows, int nb_k, int tiles, int32_t* __restrict__ hist,
-                     int32_t* __restrict__ tile_sum, int32_t* __restrict__ row_offsets) {
+                     int32_t* __restrict__ tile_sum, int32_t* __restrict__ row_offsets,
+                     int32_t* __restrict__ mix_sum) {
   __shared__ int scan_smem[33];
   __shared__ int buf[kScanBufInts];
+  if (threadIdx.x == 0) *mix_sum = 0;  // summed by head_mix_kernel, two launches later
   const int total = cta_exclusive_scan_inplace(tile_sum, tiles, scan_smem, buf);
   if (threadIdx.x == 0) row_offsets[rows] = total;
   cta_exclusive_scan_inplace(hist, (nb_k + 1) * tiles, scan_smem, buf);
@@ -299,6 +301,68 @@ __global__ void __launch_bounds__(kTileRows)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Head-major schedule.  The count order above interleaves heads wherever their
+// rows have similar counts; then the query tiles in flight at one time read
+// the K and V of many heads, which do not fit in L2 together (top-p masks at
+// HunyuanVideo 768p: 20 of 24 heads per wave of 148 tiles, 139 GB of DRAM
+// reads per forward).  So the mean number of distinct heads over the order's
+// full windows of kMixWindow entries (one wave of a B200) is measured, and
+// when it exceeds kMixHeads the schedule becomes count-descending within each
+// head, heads in order (ties by row id, as above).
+// ---------------------------------------------------------------------------
+constexpr int kMixWindow = 148;
+constexpr int kMixHeads = 8;
+constexpr int kMixMaxHeads = 8192;    // bitmap of one window: 1 KB of shared memory per warp
+constexpr int kMixMaxRowsPerHead = 8192;
+constexpr int kMixWarps = 8;
+
+// One warp per window: the window's heads as bits of a shared-memory bitmap,
+// their popcount added to *mix_sum.
+__global__ void __launch_bounds__(kMixWarps * 32)
+    head_mix_kernel(const int32_t* __restrict__ schedule, int nb_q, int heads, int windows,
+                    int32_t* __restrict__ mix_sum) {
+  __shared__ uint32_t seen[kMixWarps][kMixMaxHeads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int w = blockIdx.x * kMixWarps + warp;
+  if (w >= windows) return;
+  const int words = (heads + 31) / 32;
+  uint32_t* bm = seen[warp];
+  for (int i = lane; i < words; i += 32) bm[i] = 0u;
+  __syncwarp();
+  for (int i = lane; i < kMixWindow; i += 32) {
+    const int h = schedule[w * kMixWindow + i] / nb_q;
+    atomicOr(&bm[h >> 5], 1u << (h & 31));
+  }
+  __syncwarp();
+  int distinct = 0;
+  for (int i = lane; i < words; i += 32) distinct += __popc(bm[i]);
+  for (int o = 16; o > 0; o >>= 1) distinct += __shfl_xor_sync(0xffffffffu, distinct, o);
+  if (lane == 0) atomicAdd(mix_sum, distinct);
+}
+
+// One CTA per head, only when the windows mixed more than kMixHeads heads on
+// average: the head's rows ranked by (count descending, row ascending) by
+// counting, for every row, the rows of the head that go before it.
+__global__ void __launch_bounds__(1024)
+    head_major_kernel(const int32_t* __restrict__ counts, int nb_q, int windows,
+                      const int32_t* __restrict__ mix_sum, int32_t* __restrict__ schedule) {
+  if (*mix_sum <= kMixHeads * windows) return;  // the count order keeps few heads per wave
+  extern __shared__ int32_t head_counts[];     // nb_q
+  const int64_t base = int64_t(blockIdx.x) * nb_q;
+  for (int i = threadIdx.x; i < nb_q; i += blockDim.x) head_counts[i] = counts[base + i];
+  __syncthreads();
+  for (int i = threadIdx.x; i < nb_q; i += blockDim.x) {
+    const int c = head_counts[i];
+    int rank = 0;
+    for (int k = 0; k < nb_q; ++k) {
+      const int ck = head_counts[k];
+      rank += (ck > c) | ((ck == c) & (k < i));
+    }
+    schedule[base + rank] = int32_t(base + i);
+  }
+}
+
 // One warp per row.  The row's words are loaded one per lane, then taken one
 // at a time (broadcast by shuffle): lane j owns key block 32*w + j and, if the
 // bit is set, writes it at the row's running offset plus the number of set
@@ -327,10 +391,10 @@ __global__ void __launch_bounds__(256) write_lists_kernel(const uint32_t* __rest
 
 int num_tiles(int64_t rows) { return int((rows + kTileRows - 1) / kTileRows); }
 
-// Workspace ints: the (count, tile) table and the tile sums.
+// Workspace ints: the (count, tile) table, the tile sums and the head-mix sum.
 int64_t workspace_ints(int64_t rows, int nb_k) {
   const int64_t tiles = num_tiles(rows);
-  return (int64_t(nb_k) + 1) * tiles + tiles;
+  return (int64_t(nb_k) + 1) * tiles + tiles + 1;
 }
 
 // Grid of the row-parallel launches: kRowWarps warps per block, one row per
@@ -360,13 +424,14 @@ bsa_status check_pack_args(int B, int H, int nb_q, int nb_k, const void* bits,
 // `scratch` holds workspace_ints(rows, nb_k) ints; its contents on entry do
 // not matter (every entry is written before it is read).
 bsa_status launch_offsets_schedule_lists(const uint32_t* bits, const int32_t* counts, int rows,
-                                         int nb_k, int words, int32_t* row_offsets,
+                                         int nb_q, int nb_k, int words, int32_t* row_offsets,
                                          int32_t* col_idx, int32_t* schedule, int32_t* scratch,
                                          cudaStream_t s) {
   const int tiles = num_tiles(rows);
   const int bins = nb_k + 1;
   int32_t* table = scratch;                       // [bins][tiles]
   int32_t* tile_sum = scratch + size_t(bins) * tiles;  // [tiles]
+  int32_t* mix_sum = tile_sum + tiles;                 // [1]
   const size_t bins_bytes = size_t(bins) * sizeof(int32_t);
   const size_t ranks_bytes = size_t(kTileWarps + 1) * bins_bytes;
   const bool parallel_ranks = ranks_bytes <= kMaxDynamicSmem;
@@ -385,7 +450,8 @@ bsa_status launch_offsets_schedule_lists(const uint32_t* bits, const int32_t* co
   tile_hist_kernel<<<tiles, kTileRows, bins_bytes, s>>>(counts, rows, nb_k, tiles, table,
                                                        tile_sum);
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
-  tile_scan_kernel<<<1, kTileRows, 0, s>>>(rows, nb_k, tiles, table, tile_sum, row_offsets);
+  tile_scan_kernel<<<1, kTileRows, 0, s>>>(rows, nb_k, tiles, table, tile_sum, row_offsets,
+                                           mix_sum);
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
   if (parallel_ranks)
     tile_place_kernel<true><<<tiles, kTileRows, place_bytes, s>>>(
@@ -394,6 +460,18 @@ bsa_status launch_offsets_schedule_lists(const uint32_t* bits, const int32_t* co
     tile_place_kernel<false><<<tiles, kTileRows, place_bytes, s>>>(
         counts, rows, nb_k, tiles, table, tile_sum, row_offsets, schedule);
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
+  const int heads = rows / nb_q, windows = rows / kMixWindow;
+  if (windows > 0 && heads <= kMixMaxHeads && nb_q <= kMixMaxRowsPerHead) {
+    head_mix_kernel<<<(windows + kMixWarps - 1) / kMixWarps, kMixWarps * 32, 0, s>>>(
+        schedule, nb_q, heads, windows, mix_sum);
+    if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
+    const size_t head_bytes = size_t(nb_q) * sizeof(int32_t);
+    if (cudaFuncSetAttribute(head_major_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(head_bytes)) != cudaSuccess)
+      return BSA_ERR_LAUNCH;
+    head_major_kernel<<<heads, 1024, head_bytes, s>>>(counts, nb_q, windows, mix_sum, schedule);
+    if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
+  }
   if (col_idx) {
     write_lists_kernel<<<row_grid(rows), 256, 0, s>>>(bits, rows, words, row_offsets, col_idx);
     if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
@@ -410,10 +488,10 @@ size_t bsa::pack_scratch_bytes(int64_t rows, int nb_k) {
   return (bytes + 255) & ~size_t(255);
 }
 
-bsa_status bsa::pack_finish(const uint32_t* bits, const int32_t* counts, int rows, int nb_k,
-                            int32_t* row_offsets, int32_t* col_idx, int32_t* schedule,
+bsa_status bsa::pack_finish(const uint32_t* bits, const int32_t* counts, int rows, int nb_q,
+                            int nb_k, int32_t* row_offsets, int32_t* col_idx, int32_t* schedule,
                             void* scratch, cudaStream_t s) {
-  return launch_offsets_schedule_lists(bits, counts, rows, nb_k, (nb_k + 31) / 32, row_offsets,
+  return launch_offsets_schedule_lists(bits, counts, rows, nb_q, nb_k, (nb_k + 31) / 32, row_offsets,
                                        col_idx, schedule, static_cast<int32_t*>(scratch), s);
 }
 
@@ -440,7 +518,7 @@ extern "C" bsa_status bsa_pack_mask(const uint8_t* dense, int B, int H, int nb_q
   const int words = (nb_k + 31) / 32;
   pack_rows_kernel<<<row_grid(rows), 256, 0, s>>>(dense, rows, nb_k, words, bits, counts);
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
-  return launch_offsets_schedule_lists(bits, counts, rows, nb_k, words, row_offsets, col_idx,
+  return launch_offsets_schedule_lists(bits, counts, rows, nb_q, nb_k, words, row_offsets, col_idx,
                                        schedule, static_cast<int32_t*>(workspace), s);
 }
 
@@ -466,7 +544,7 @@ extern "C" bsa_status bsa_pack_mask_from_threshold(const float* thr, const float
   pack_threshold_rows_kernel<<<row_grid(rows), 256, 0, s>>>(thr, p, nb_q, H * nb_q, rows, nb_k,
                                                             words, bits, counts);
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
-  return launch_offsets_schedule_lists(bits, counts, rows, nb_k, words, row_offsets, col_idx,
+  return launch_offsets_schedule_lists(bits, counts, rows, nb_q, nb_k, words, row_offsets, col_idx,
                                        schedule, static_cast<int32_t*>(workspace), s);
 }
 
@@ -527,6 +605,6 @@ extern "C" bsa_status bsa_pack_mask_noalloc(const uint8_t* dense, int B, int H, 
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
   // every scratch entry the sort reads is written earlier in the same call, so
   // whatever an earlier call left there does not matter
-  return launch_offsets_schedule_lists(bits, counts, rows, nb_k, words, row_offsets, col_idx,
+  return launch_offsets_schedule_lists(bits, counts, rows, nb_q, nb_k, words, row_offsets, col_idx,
                                        schedule, scratch, s);
 }

@@ -341,6 +341,6 @@ extern "C" bsa_status bsa_predict_top_p(const void* q, const void* k, int B, int
   else
     st = launch_score<64>(grid, smem, s, qbar, kbar, H, nb, d, tau, top_p, bits, counts);
   if (st != BSA_OK) return st;
-  return bsa::pack_finish(bits, counts, int(BH * nb), nb, row_offsets, col_idx, schedule, scratch,
+  return bsa::pack_finish(bits, counts, int(BH * nb), nb, nb, row_offsets, col_idx, schedule, scratch,
                           s);
 }

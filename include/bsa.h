@@ -56,7 +56,7 @@ typedef struct {
   const int32_t* counts;       /* [B, H, nb_q] kept key blocks per query block */
   const int32_t* row_offsets;  /* [B*H*nb_q + 1] exclusive prefix of counts */
   const int32_t* col_idx;      /* [row_offsets[B*H*nb_q]] ascending kept key blocks per row */
-  const int32_t* schedule;     /* [B*H*nb_q] flat row ids, most kept blocks first, stable */
+  const int32_t* schedule;     /* [B*H*nb_q] flat row ids in work order (see bsa_pack_mask) */
   int B, H, nb_q, nb_k, words;
 } bsa_mask;
 
@@ -83,6 +83,14 @@ const char* bsa_status_string(bsa_status status);
  *               row_offsets[r+1]).  May be NULL to skip the lists.
  *   schedule    out [B*H*nb_q] int32 flat row ids r = (b*H + h)*nb_q + i,
  *               ordered by counts descending; equal counts keep ascending r.
+ *               Then the order is checked for how many heads it mixes: over
+ *               its full windows of 148 consecutive entries (one wave of a
+ *               B200), if the distinct heads h' = r / nb_q (one per (b, h))
+ *               total more than 8 per window, the schedule is instead ordered
+ *               by head h' ascending, then counts descending, then r
+ *               ascending.  (Query tiles taken together then share one head's
+ *               K and V in L2; the check is skipped, keeping the count
+ *               order, when B*H > 8192 or nb_q > 8192.)
  *   workspace   device scratch of at least bsa_pack_mask_workspace(...) bytes,
  *               16-byte aligned; its contents on entry do not matter.
  *
@@ -110,7 +118,7 @@ bsa_status bsa_pack_mask(const uint8_t* dense, int B, int H, int nb_q, int nb_k,
  * that loads it until the process exits.
  *
  * Limit: the built-in scratch holds 131072 ints and the call needs
- * (nb_k + 2) * ceil(B*H*nb_q / 1024) of them (e.g. every workload with up to
+ * (nb_k + 2) * ceil(B*H*nb_q / 1024) + 1 of them (e.g. every workload with up to
  * 40 heads of 1024 query blocks of 1024 key blocks, B = 1, fits); a larger
  * call returns BSA_ERR_WORKSPACE (use bsa_pack_mask).  The first call on each device
  * looks up the array's device address (cudaGetSymbolAddress) with that device

@@ -14,6 +14,7 @@ Intrinsic Sparse Attention Topology for Video Diffusion Transformers"):
                             Appendix E, Algorithm 2 (base + CTZ).
 - ``crm_lists``          -- Appendix E, Algorithm 2 (Init/Advance/Next/Index).
 - ``schedule``           -- rows by kept-block count, largest first, stable
+                              (head-major when that order mixes many heads)
                             (the pages are silent; plainest reading).
 - ``tile_order``, ``permute``, ``unpermute``
                          -- token reordering into 3-D tiles, Sec. 5.4 and 5.5.
@@ -78,7 +79,7 @@ def _load():
             lib.oracle_pack_bits.argtypes = [P, I64, I, P]
             lib.oracle_crm_lists.argtypes = [P, I64, I, P, P, P]
             lib.oracle_crm_lists.restype = I64
-            lib.oracle_schedule.argtypes = [P, I64, P]
+            lib.oracle_schedule.argtypes = [P, I64, I64, P]
             lib.oracle_tile_order.argtypes = [I, I, I, I, I, I, P]
             lib.oracle_permute.argtypes = [P, P, I64, I64, I64, I, P]
             lib.oracle_unpermute.argtypes = [P, P, I64, I64, I64, I, P]
@@ -137,10 +138,13 @@ def crm_lists(bits: np.ndarray):
     return counts, offsets, col_idx[:total]
 
 
-def schedule(counts: np.ndarray) -> np.ndarray:
+def schedule(counts: np.ndarray, nb_q: int = 0) -> np.ndarray:
+    """Work order of the rows: by count, largest first, stable; with nb_q > 0
+    (rows per head) the head-major form when the count order mixes more than 8
+    heads per window of 148 entries (see oracle.c)."""
     counts = np.ascontiguousarray(counts, dtype=np.int32)
     out = np.zeros(counts.size, dtype=np.int32)
-    _load().oracle_schedule(_ptr(counts), counts.size, _ptr(out))
+    _load().oracle_schedule(_ptr(counts), counts.size, int(nb_q), _ptr(out))
     return out
 
 

@@ -19,7 +19,7 @@ def _pack_and_compare(dense: np.ndarray):
     torch.cuda.synchronize()
     bits_ref = oracle.pack_bits(dense)
     counts_ref, offsets_ref, col_ref = oracle.crm_lists(bits_ref)
-    sched_ref = oracle.schedule(counts_ref)
+    sched_ref = oracle.schedule(counts_ref, nbq)
     np.testing.assert_array_equal(pm.bits.cpu().numpy().view(np.uint32), bits_ref)
     np.testing.assert_array_equal(pm.counts.cpu().numpy(), counts_ref)
     np.testing.assert_array_equal(pm.row_offsets.cpu().numpy().astype(np.int64), offsets_ref)
@@ -32,6 +32,42 @@ def _pack_and_compare(dense: np.ndarray):
 def test_pack_mask_workloads(cuda_ok, name):
     w = I.WORKLOADS[name]
     _pack_and_compare(I.gen_mask(w))
+
+
+def _mask_with_counts(counts_per_row: np.ndarray, nbk: int, seed: int) -> np.ndarray:
+    """[1, H, nbq, nbk] mask whose row (h, i) keeps counts_per_row[h, i] random blocks."""
+    rng = np.random.default_rng(seed)
+    H, nbq = counts_per_row.shape
+    dense = np.zeros((1, H, nbq, nbk), dtype=np.uint8)
+    for h in range(H):
+        for i in range(nbq):
+            dense[0, h, i, rng.choice(nbk, size=int(counts_per_row[h, i]), replace=False)] = 1
+    return dense
+
+
+def test_pack_schedule_head_major_when_heads_mix(cuda_ok):
+    # every head draws its counts from one distribution: the count order mixes
+    # all 16 heads in every window of 148, so the schedule goes head-major
+    rng = np.random.default_rng(11)
+    counts = rng.integers(0, 200, size=(16, 96))
+    dense = _mask_with_counts(counts, 256, 12)
+    _pack_and_compare(dense)
+    B, H, nbq, nbk = dense.shape
+    sched = oracle.schedule(oracle.crm_lists(oracle.pack_bits(dense))[0], nbq)
+    assert np.all(np.diff(sched // nbq) >= 0)  # the head-major form was taken
+
+
+@pytest.mark.parametrize("heads,expect_head_major", [(8, False), (9, True)])
+def test_pack_schedule_mix_threshold(cuda_ok, heads, expect_head_major):
+    # row i of every head keeps 200 - i blocks: each count level lists all the
+    # heads, so every window of 148 holds all of them; 8 heads per window stays
+    # in count order, 9 is more than 8 and turns head-major
+    nbq = 148
+    counts = np.tile(200 - np.arange(nbq), (heads, 1))
+    dense = _mask_with_counts(counts, 256, 13)
+    _pack_and_compare(dense)
+    sched = oracle.schedule(oracle.crm_lists(oracle.pack_bits(dense))[0], nbq)
+    assert bool(np.all(np.diff(sched // nbq) >= 0)) == expect_head_major
 
 
 @pytest.mark.parametrize("shape,density", [((1, 1, 1, 1), 1.0), ((1, 3, 5, 33), 0.3),

@@ -23,7 +23,7 @@ pytestmark = pytest.mark.gpu
 def _oracle_pack(dense):
     bits = oracle.pack_bits(dense)
     counts, offsets, cols = oracle.crm_lists(bits)
-    return bits, counts, offsets, cols, oracle.schedule(counts)
+    return bits, counts, offsets, cols, oracle.schedule(counts, dense.shape[2])
 
 
 def _compare(pm, ref):

@@ -86,6 +86,52 @@ def test_schedule_is_stable_count_descending():
     np.testing.assert_array_equal(sched, np.array(expect, dtype=np.int32))
 
 
+def test_schedule_head_major_when_the_count_order_mixes_heads():
+    # 16 heads drawing counts from one distribution: every window of 148 holds
+    # about all 16 heads, so the order is head by head, count order inside
+    rng = np.random.default_rng(6)
+    nb_q = 96
+    counts = rng.integers(0, 200, size=16 * nb_q).astype(np.int32)
+    sched = oracle.schedule(counts, nb_q)
+    expect = sorted(range(counts.size), key=lambda r: (r // nb_q, -int(counts[r]), r))
+    np.testing.assert_array_equal(sched, np.array(expect, dtype=np.int32))
+
+
+def test_schedule_stays_count_order_when_heads_separate():
+    # disjoint count ranges per head: the count order is already head by head
+    # in reverse, a few heads per window, and is kept as it is
+    rng = np.random.default_rng(7)
+    nb_q = 96
+    counts = np.concatenate([h * 300 + rng.integers(0, 250, size=nb_q) for h in range(16)])
+    counts = counts.astype(np.int32)
+    sched = oracle.schedule(counts, nb_q)
+    expect = sorted(range(counts.size), key=lambda r: (-int(counts[r]), r))
+    np.testing.assert_array_equal(sched, np.array(expect, dtype=np.int32))
+
+
+@pytest.mark.parametrize("heads,head_major", [(8, False), (9, True)])
+def test_schedule_mix_threshold_is_more_than_eight_heads(heads, head_major):
+    # row i of each head has count 200 - i: each count level lists every head,
+    # so each window of 148 holds all heads; 8 per window keeps the count
+    # order, 9 (more than 8) switches
+    nb_q = 148
+    counts = np.tile(200 - np.arange(nb_q), heads).astype(np.int32)
+    sched = oracle.schedule(counts, nb_q)
+    if head_major:
+        key = lambda r: (r // nb_q, -int(counts[r]), r)
+    else:
+        key = lambda r: (-int(counts[r]), r)
+    np.testing.assert_array_equal(sched, np.array(sorted(range(counts.size), key=key), np.int32))
+
+
+def test_schedule_short_or_single_head_keeps_count_order():
+    rng = np.random.default_rng(8)
+    for counts, nb_q in ((rng.integers(0, 9, size=100), 10), (rng.integers(0, 9, size=600), 600)):
+        counts = counts.astype(np.int32)
+        expect = sorted(range(counts.size), key=lambda r: (-int(counts[r]), r))
+        np.testing.assert_array_equal(oracle.schedule(counts, nb_q), np.array(expect, np.int32))
+
+
 # ---------------------------------------------------------------- tile order
 def test_tile_order_divisible_matches_reshape():
     T, Hs, Ws, tt, th, tw = 4, 16, 16, 2, 8, 4
