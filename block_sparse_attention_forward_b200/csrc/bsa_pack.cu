@@ -1,11 +1,11 @@
 // bsa_pack.cu -- per-head block masks -> CRM rows, counts, row offsets,
-// ascending key-block lists and the count-ordered schedule.
+// ascending key-block lists and the schedule (the forward's work order).
 //
 // CRM layout ("ScalingAttention", Sec. 4.3.2 and Appendix E, Algorithm 2): one
 // row of uint32 words per query block; bit j of word w is key block 32*w + j
 // (the iterator's base grows by 32 per word and the index is base + CTZ).
 //
-// Five launches on the caller's stream:
+// Seven launches on the caller's stream (five below one window of rows):
 //   1. rows:        one warp per row; a coalesced read of the row per word,
 //                   __ballot_sync builds the word, popcounts sum.  Two
 //                   variants: a dense uint8 mask (bsa_pack_mask), or a
@@ -22,7 +22,10 @@
 //   4. tile_place:  one CTA per tile; row_offsets from a block scan, then the
 //                   tile's warps take turns placing their rows at their
 //                   count's next slot -- in row order, so the sort is stable.
-//   5. write_lists: one warp per row; words are taken one at a time and each
+//   5. head_mix:    distinct heads per window of 148 entries of that order.
+//   6. head_major:  if they exceed 8 per window on average, the schedule
+//                   becomes count-descending within each head, heads in order.
+//   7. write_lists: one warp per row; words are taken one at a time and each
 //                   lane writes its key block at the row's running offset, so
 //                   each store instruction writes consecutive addresses.
 #include <cuda_runtime.h>
