@@ -57,6 +57,21 @@ def test_pack_schedule_head_major_when_heads_mix(cuda_ok):
     assert np.all(np.diff(sched // nbq) >= 0)  # the head-major form was taken
 
 
+def test_pack_schedule_head_major_long_heads_and_batches(cuda_ok):
+    # B = 2 (each (b, h) is its own head in the rule) and 1,500 rows per head:
+    # more rows than one CTA's threads, so the head-major ranking loops
+    import block_sparse_attention_forward_b200 as bsa
+    rng = np.random.default_rng(14)
+    B, H, nbq, nbk = 2, 5, 1500, 256
+    dense = (rng.random((B, H, nbq, nbk)) < rng.uniform(0.1, 0.9, size=(B, H, nbq, 1))).astype(np.uint8)
+    pm = bsa.pack_mask(torch.from_numpy(dense).cuda())
+    torch.cuda.synchronize()
+    counts = oracle.crm_lists(oracle.pack_bits(dense))[0]
+    sched = oracle.schedule(counts, nbq)
+    assert np.all(np.diff(sched // nbq) >= 0)  # ten heads mix: head-major taken
+    np.testing.assert_array_equal(pm.schedule.cpu().numpy(), sched)
+
+
 @pytest.mark.parametrize("heads,expect_head_major", [(8, False), (9, True)])
 def test_pack_schedule_mix_threshold(cuda_ok, heads, expect_head_major):
     # row i of every head keeps 200 - i blocks: each count level lists all the
