@@ -24,7 +24,8 @@
 //                   count's next slot -- in row order, so the sort is stable.
 //   5. head_mix:    distinct heads per window of 148 entries of that order.
 //   6. head_major:  if they exceed 8 per window on average, the schedule
-//                   becomes count-descending within each head, heads in order.
+//                   becomes count-descending within each head, heads in order
+//                   (a counting sort per head, one CTA each).
 //   7. write_lists: one warp per row; words are taken one at a time and each
 //                   lane writes its key block at the row's running offset, so
 //                   each store instruction writes consecutive addresses.
@@ -344,25 +345,54 @@ __global__ void __launch_bounds__(kMixWarps * 32)
   if (lane == 0) atomicAdd(mix_sum, distinct);
 }
 
-// One CTA per head, only when the windows mixed more than kMixHeads heads on
-// average: the head's rows ranked by (count descending, row ascending) by
-// counting, for every row, the rows of the head that go before it.
-__global__ void __launch_bounds__(1024)
-    head_major_kernel(const int32_t* __restrict__ counts, int nb_q, int windows,
+// One CTA per head (kTileRows threads), only when the windows mixed more than
+// kMixHeads heads on average: a counting sort of the head's rows by count,
+// descending.  Histogram of keys d = nb_k - count in shared memory, exclusive
+// scan of it (chunks of kTileRows bins), then the rows in order, a chunk of
+// kTileRows at a time, the chunk's warps taking turns: each lane's slot is
+// its key's next slot plus the lanes before it with the same key, so equal
+// counts keep ascending row order.
+__global__ void __launch_bounds__(kTileRows)
+    head_major_kernel(const int32_t* __restrict__ counts, int nb_q, int nb_k, int windows,
                       const int32_t* __restrict__ mix_sum, int32_t* __restrict__ schedule) {
   if (*mix_sum <= kMixHeads * windows) return;  // the count order keeps few heads per wave
-  extern __shared__ int32_t head_counts[];     // nb_q
+  extern __shared__ int32_t next_slot[];        // nb_k + 1 bins
+  __shared__ int scan_smem[33];
+  const int bins = nb_k + 1;
   const int64_t base = int64_t(blockIdx.x) * nb_q;
-  for (int i = threadIdx.x; i < nb_q; i += blockDim.x) head_counts[i] = counts[base + i];
+  for (int d = threadIdx.x; d < bins; d += kTileRows) next_slot[d] = 0;
   __syncthreads();
-  for (int i = threadIdx.x; i < nb_q; i += blockDim.x) {
-    const int c = head_counts[i];
-    int rank = 0;
-    for (int k = 0; k < nb_q; ++k) {
-      const int ck = head_counts[k];
-      rank += (ck > c) | ((ck == c) & (k < i));
+  for (int i = threadIdx.x; i < nb_q; i += kTileRows) atomicAdd(&next_slot[nb_k - counts[base + i]], 1);
+  __syncthreads();
+  int carry = 0;
+  for (int d0 = 0; d0 < bins; d0 += kTileRows) {
+    const int d = d0 + int(threadIdx.x);
+    const int x = d < bins ? next_slot[d] : 0;
+    int chunk_total;
+    const int pre = block_exclusive_scan(x, scan_smem, &chunk_total);
+    if (d < bins) next_slot[d] = carry + pre;
+    carry += chunk_total;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned below = (1u << lane) - 1u;
+  const int key_bits = 32 - __clz(nb_k);
+  for (int i0 = 0; i0 < nb_q; i0 += kTileRows) {
+    const int i = i0 + int(threadIdx.x);
+    const bool active = i < nb_q;
+    const unsigned act = __ballot_sync(0xffffffffu, active);
+    const int d = active ? nb_k - counts[base + i] : 0;
+    for (int w = 0; w < kTileWarps; ++w) {
+      if (warp == w && active) {
+        const unsigned peers = equal_keys(act, d, key_bits);
+        const int rank = __popc(peers & below);
+        const int pos = next_slot[d] + rank;
+        schedule[base + pos] = int32_t(base + i);
+        __syncwarp(act);
+        if (rank == 0) next_slot[d] = pos + __popc(peers);
+      }
+      __syncthreads();
     }
-    schedule[base + rank] = int32_t(base + i);
   }
 }
 
@@ -468,11 +498,11 @@ bsa_status launch_offsets_schedule_lists(const uint32_t* bits, const int32_t* co
     head_mix_kernel<<<(windows + kMixWarps - 1) / kMixWarps, kMixWarps * 32, 0, s>>>(
         schedule, nb_q, heads, windows, mix_sum);
     if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
-    const size_t head_bytes = size_t(nb_q) * sizeof(int32_t);
     if (cudaFuncSetAttribute(head_major_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(head_bytes)) != cudaSuccess)
+                             int(bins_bytes)) != cudaSuccess)
       return BSA_ERR_LAUNCH;
-    head_major_kernel<<<heads, 1024, head_bytes, s>>>(counts, nb_q, windows, mix_sum, schedule);
+    head_major_kernel<<<heads, kTileRows, bins_bytes, s>>>(counts, nb_q, nb_k, windows, mix_sum,
+                                                          schedule);
     if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
   }
   if (col_idx) {
