@@ -634,7 +634,8 @@ def main():
         e2e = {"value": total_flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "call": "bsa_attention_host (pinned host buffers, heads in chunks of "
-                       f"{-(-w.B * w.H // 16)}, copies overlapped with the kernels)",
+                       f"{-(-w.B * w.H // 16)} with one-head first and last chunks, copies "
+                       "overlapped with the kernels)",
                "bound": "host-to-device copy of q, k, v and mask (PCIe)"}
         del sp
 

@@ -20,6 +20,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <vector>
 
 #include "bsa.h"
 #include "bsa_internal.h"
@@ -160,12 +161,25 @@ extern "C" bsa_status bsa_attention_host(const void* q, const void* k, const voi
   char* ws = static_cast<char*>(workspace);
   const size_t head_frame = size_t(n) * d * 2, head_mask = size_t(nb) * nb;
   const size_t head_lse = size_t(n_pad) * 4;
-  const int chunks = (BH + hc - 1) / hc;
+  // Chunk boundaries: with room for it, the first and the last chunk hold one
+  // head each, so that the pipeline fills (the first copy-in before any
+  // kernel) and drains (the last kernels and copy-out after the last copy-in)
+  // in one head's time; the chunks between hold hc heads.
+  std::vector<int> start{0};
+  if (hc > 1 && BH > 2) {
+    start.push_back(1);
+    for (int h = 1 + hc; h < BH - 1; h += hc) start.push_back(h);
+    start.push_back(BH - 1);
+  } else {
+    for (int h = hc; h < BH; h += hc) start.push_back(h);
+  }
+  start.push_back(BH);
+  const int chunks = int(start.size()) - 1;
   auto ok = [](cudaError_t e) { return e == cudaSuccess; };
   for (int c = 0; c < chunks; ++c) {
     const int s = c % kSlots;
     char* base = ws + size_t(s) * L.bytes;
-    const int h0 = c * hc, hn = hc < BH - h0 ? hc : BH - h0;
+    const int h0 = start[c], hn = start[c + 1] - start[c];
     // ---- copy in (waits until chunk c - 2 has finished reading this slot)
     if (c >= kSlots && !ok(cudaStreamWaitEvent(ctx->copy_in, ctx->comp_done[s], 0)))
       return BSA_ERR_LAUNCH;

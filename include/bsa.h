@@ -354,9 +354,11 @@ bsa_status bsa_forward_blocks(const void* q, const void* k, const void* v, const
  * kernels.
  *
  * Heads are independent (each has its own mask, token order and softmax), so
- * the B*H heads run in chunks of heads_per_chunk (<= 0: ceil(B*H / 16)) as a
- * three-stage pipeline: chunk c + 1 is copied in and chunk c - 1 copied out
- * while chunk c computes on `stream`.  Two auxiliary streams per device (made
+ * the B*H heads run in chunks of at most heads_per_chunk (<= 0: ceil(B*H / 16))
+ * as a three-stage pipeline: chunk c + 1 is copied in and chunk c - 1 copied
+ * out while chunk c computes on `stream`.  When heads_per_chunk > 1 and
+ * B*H > 2, the first and the last chunk hold one head each, so the pipeline
+ * fills and drains in one head's time.  Two auxiliary streams per device (made
  * on first use) carry the copies; they start after the work already queued on
  * `stream` and are joined back into it, so the call is ordered on `stream`
  * like any other.  Calls on one device from several host threads at once
