@@ -9,21 +9,28 @@ bsa_tile_permute of q, k, v, bsa_forward, bsa_tile_unpermute of the output.
 metric: effective TFLOPS = 4 * d * block^2 * (kept tiles) / time, with the
 step time as denominator for `value` and the forward kernel's own time for
 `roofline.achieved`.  Inputs (3 x 774 MB for the default workload) are larger
-than L2, so no flush is needed between steps.
+than L2, so no flush is needed between steps.  The forward is timed per launch
+with CUDA events, so its roofline fraction is taken against the burst bf16
+peak; the line also gives it against the sustained peak and against the burst
+peak scaled to the median SM clock seen during the timed steps.
 
-With N > 1 (torchrun), every rank runs its own independent problem of the same
-shape (different seed): the path shards by (batch, head) with no exchange, so
-there is no collective on the data path (weak scaling); the step time is the
-max over ranks.
+With N > 1 (torchrun), the ranks split ONE problem of the workload by flat
+head index (sharding.head_range): every rank packs, permutes and attends its
+own heads, with no exchange between ranks (the heads are independent), so
+there is no collective on the data path; the step time is the max over ranks
+and `value` counts the whole problem's kept tiles (strong scaling).
 
 After the timed steps, `next_rows` reports further steps measured on their own
-(L2 flushed before each call): bsa_pack_mask_from_threshold at the workload's
-block grid, bsa_threshold_resize of a 480p-grid map to it, bsa_gather_rows
-applying the Hilbert-curve order and head-aware tile orders to one tensor,
-the online top-p predictor bsa_predict_top_p on the workload's q and k, the
-forward with 64-token key blocks under 128-token query blocks, and the forward
-on an all-ones mask (the speedup of the workload's mask over it; PyTorch's dense
-SDPA on the same tensors as context).
+(L2 flushed before each call): bsa_tile_permute and bsa_tile_unpermute of one
+tensor, bsa_pack_mask_from_threshold at the workload's block grid,
+bsa_threshold_resize of a 480p-grid map to it, bsa_gather_rows applying the
+Hilbert-curve order and head-aware tile orders to one tensor, the online top-p
+predictor bsa_predict_top_p on the workload's q and k, the forward with 64-token
+key blocks under 128-token query blocks, the forward on an all-ones mask (the
+speedup of the workload's mask over it, and a density sweep), PyTorch's dense
+SDPA on the same tensors as context, and `by_length`: the masked forward, the
+all-ones forward and dense SDPA on each of the four full-size workloads
+(32,760 to 126,720 tokens).
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of query blocks of the same workload (rank 0 only).
@@ -470,13 +477,106 @@ def measure_dense_rows(w, dev, stream, peak_tflops: float, sparse_fwd_ms: float 
     return res
 
 
-def workload_config(w, mask):
+def measure_permute_row(w, dev, stream, hbm_gbs: float, x_dev: torch.Tensor):
+    """bsa_tile_permute and bsa_tile_unpermute of one [B, H, N, d] bf16 tensor of the
+    workload, each launch timed alone with CUDA events, L2 flushed before each call.
+    HBM-bound; algorithmic bytes = N rows read + n_pad rows written per head
+    (permute) and n_pad rows read + N rows written (unpermute): one read and one
+    write of the tensor."""
+    import block_sparse_attention_forward_b200 as bsa
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    grid, tile = (w.T, w.Hs, w.Ws), (w.tt, w.th, w.tw)
+    yp = torch.empty((w.B, w.H, w.n_pad, w.d), dtype=torch.bfloat16, device=dev)
+    back = torch.empty_like(x_dev)
+    nbytes = w.B * w.H * (w.n + w.n_pad) * w.d * 2
+    res = {}
+    for name, fn in (("tile_permute", lambda: bsa.tile_permute(x_dev, grid, tile, w.n_pad, out=yp)),
+                     ("tile_unpermute", lambda: bsa.tile_unpermute(yp, grid, tile, out=back))):
+        us = time_device_us(fn, stream, flush)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        res[name] = {"us": us, "bytes": nbytes, "achieved_gbs": gbs, "frac_hbm": gbs / hbm_gbs,
+                     "bound": "hbm", "launches": 1, "l2": "flushed before each call"}
+    if not torch.equal(back, x_dev):
+        raise RuntimeError("tile_unpermute(tile_permute(x)) != x")
+    del flush, yp, back
+    return {"permute": res}
+
+
+def measure_by_length(dev, stream, peak_tflops: float, reuse=None):
+    """The pages' kernel benchmark over sequence lengths: for each full-size
+    workload, the masked forward (its own mask), the forward on an all-ones mask and
+    PyTorch's dense SDPA (context, not ours) on the same permuted tensors, each a
+    short loop with the L2 flushed before every call.  `reuse` = (workload name, qp,
+    kp, vp, packed mask, mask) skips regenerating the timed workload's inputs."""
+    import block_sparse_attention_forward_b200 as bsa
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rows = []
+    sdpa = torch.nn.functional.scaled_dot_product_attention
+    for name in ("wan13b_480p", "wan14b_480p", "wan14b_720p", "hunyuan_768p"):
+        w = I.WORKLOADS[name]
+        if reuse is not None and reuse[0] == name:
+            qp, kp, vp, pm, mask = reuse[1:]
+        else:
+            q, k, v = I.gen_qkv(w)
+            mask = I.gen_mask(w, q, k)
+            grid, tile = (w.T, w.Hs, w.Ws), (w.tt, w.th, w.tw)
+            qp, kp, vp = (bsa.tile_permute(t.to(dev), grid, tile, w.n_pad) for t in (q, k, v))
+            del q, k, v
+            pm = bsa.pack_mask(torch.from_numpy(mask).to(dev))
+        out = torch.empty_like(qp)
+        lse = torch.empty((w.B, w.H, w.n_pad), dtype=torch.float32, device=dev)
+        kept = I.kept_tiles(mask)
+        tile_flop = 4.0 * w.d * w.block * w.block
+        us_m = time_device_us(lambda: bsa.forward(qp, kp, vp, pm, w.n, w.block, out=out, lse=lse),
+                              stream, flush, iters=5, warmup=2)
+        ones = bsa.pack_mask(torch.ones((w.B, w.H, w.nb, w.nb), dtype=torch.uint8, device=dev))
+        us_1 = time_device_us(lambda: bsa.forward(qp, kp, vp, ones, w.n, w.block, out=out,
+                                                  lse=lse), stream, flush, iters=3, warmup=1)
+        if bsa.device_error() != 0:
+            raise RuntimeError(f"device error in the forward on {name}")
+        qd, kd, vd = (t[:, :, :w.n] for t in (qp, kp, vp))
+        try:
+            us_s = time_device_us(lambda: sdpa(qd, kd, vd), stream, flush, iters=3, warmup=1)
+        except RuntimeError:
+            us_s = None
+        dense_flop = tile_flop * w.B * w.H * w.nb * w.nb
+        tf_m = tile_flop * kept / (us_m * 1e-6) / 1e12
+        rows.append({
+            "workload": name, "n_tokens": w.n, "heads": w.H, "density": kept / (w.B * w.H * w.nb * w.nb),
+            "masked_us": us_m, "masked_tflops": tf_m, "masked_frac": tf_m / peak_tflops,
+            "all_ones_us": us_1, "all_ones_tflops": dense_flop / (us_1 * 1e-6) / 1e12,
+            "sdpa_us": us_s,
+            "sdpa_tflops": (4.0 * w.d * w.n * w.n * w.B * w.H / (us_s * 1e-6) / 1e12) if us_s else None,
+            "all_ones_over_sdpa": (us_1 / us_s) if us_s else None,
+            "masked_speedup_vs_all_ones": us_1 / us_m,
+        })
+        del qp, kp, vp, pm, ones, out, lse, qd, kd, vd
+        torch.cuda.empty_cache()
+    del flush
+    return {"by_length": rows, "by_length_peak": peak_tflops}
+
+
+def workload_config(w, mask, world: int = 1):
     kept = I.kept_tiles(mask)
     total = w.B * w.H * w.nb * w.nb
     return {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "grid": [w.T, w.Hs, w.Ws],
             "tile": [w.tt, w.th, w.tw], "block": w.block, "n_tokens": w.n, "n_pad": w.n_pad,
             "kept_tiles": kept, "density": kept / total, "mask": w.mask_kind,
-            "l2": "inputs larger than L2 (no flush)", "parallelism": "independent problems per rank"}
+            "l2": "inputs larger than L2 (no flush)",
+            "parallelism": (f"heads split over {world} ranks (head_range), no exchange"
+                            if world > 1 else "one GPU, all heads")}
+
+
+def shard_workload(w, q, k, v, mask, world: int, rank: int):
+    """This rank's heads of one problem: flat heads [lo, hi) of B*H, as a workload
+    with B = 1 and H = hi - lo (every head is an independent problem)."""
+    import dataclasses
+
+    from block_sparse_attention_forward_b200.sharding import head_range
+    lo, hi = head_range(w.B * w.H, world, rank)
+    flat = lambda x: x.reshape(1, w.B * w.H, *x.shape[2:])[:, lo:hi].contiguous()  # noqa: E731
+    ws = dataclasses.replace(w, B=1, H=hi - lo)
+    return ws, flat(q), flat(k), flat(v), np.ascontiguousarray(flat(mask)), (lo, hi)
 
 
 def main():
@@ -492,6 +592,8 @@ def main():
                     help="skip the threshold-map rows measured after the timed steps")
     ap.add_argument("--only-next", action="store_true",
                     help="measure only the threshold-map rows (a small case for profiling)")
+    ap.add_argument("--no-by-length", action="store_true",
+                    help="skip the forward / all-ones / SDPA comparison over the four workloads")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (smaller cases for profiling captures)")
     args = ap.parse_args()
@@ -517,7 +619,7 @@ def main():
                                        float(peaks["hbm_gbs"])))
         rows.update(measure_predict_row(w, dev, torch.cuda.current_stream(dev),
                                         float(peaks["hbm_gbs"])))
-        pk = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        pk = float(peaks["bf16_tflops"])
         rows.update(measure_finer_keys_row(w, dev, torch.cuda.current_stream(dev), pk))
         rows.update(measure_dense_rows(w, dev, torch.cuda.current_stream(dev), pk, None))
         if rank == 0:
@@ -525,9 +627,11 @@ def main():
         if world > 1:
             torch.distributed.destroy_process_group()
         return 0
-    seed = w.seed + 7919 * rank
-    q, k, v = I.gen_qkv(w, seed=seed)
-    mask = I.gen_mask(w, q, k, seed=seed)
+    q_all, k_all, v_all = I.gen_qkv(w)
+    mask_all = I.gen_mask(w, q_all, k_all)
+    w_all = w
+    w, q, k, v, mask, heads = shard_workload(w_all, q_all, k_all, v_all, mask_all, world, rank)
+    del q_all, k_all, v_all
     flops = I.effective_flops(w, mask)
     grid, tile = (w.T, w.Hs, w.Ws), (w.tt, w.th, w.tw)
 
@@ -585,6 +689,7 @@ def main():
     if bsa.device_error() != 0:
         raise RuntimeError("device error during the timed region")
 
+    fwd_ms_local = fwd_ms  # this rank's forward, for the kernel's roofline
     t = torch.tensor([ms_total, fwd_ms, flops], dtype=torch.float64, device=dev)
     total_flops = flops
     if world > 1:
@@ -641,20 +746,34 @@ def main():
 
     # ---------------------------------------------------------------- roofline
     peaks, peak_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    # the forward is timed per launch (CUDA events around each call), not as a
+    # seconds-long loop: the burst peak is its denominator
+    peak = float(peaks["bf16_tflops"])
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
+    clocks = sampler.summary(t_wall0, t_wall1)
     next_rows = None
     if not args.no_next and world == 1:  # extra rows only at N = 1: no GPU held longer
-        next_rows = measure_threshold_rows(w, dev, stream, float(peaks["hbm_gbs"]))
-        next_rows.update(measure_order_rows(w, dev, stream, float(peaks["hbm_gbs"])))
-        next_rows.update(measure_predict_row(w, dev, stream, float(peaks["hbm_gbs"])))
+        hbm = float(peaks["hbm_gbs"])
+        next_rows = measure_permute_row(w, dev, stream, hbm, qd)
+        next_rows.update(measure_threshold_rows(w, dev, stream, hbm))
+        next_rows.update(measure_order_rows(w, dev, stream, hbm))
+        next_rows.update(measure_predict_row(w, dev, stream, hbm))
         next_rows.update(measure_finer_keys_row(w, dev, stream, peak))
-        next_rows.update(measure_dense_rows(w, dev, stream, peak, fwd_ms))
-    fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
+        next_rows.update(measure_dense_rows(w, dev, stream, peak, fwd_ms_local))
+        if not args.no_by_length:
+            pm_main = bsa.pack_mask(maskd)
+            next_rows.update(measure_by_length(dev, stream, peak,
+                                               reuse=(w.name, qp, kp, vp, pm_main, mask)))
+    fwd_tflops = flops / (fwd_ms_local * 1e-3) / 1e12
+    sm_mhz, sm_max = clocks.get("sm_mhz"), clocks.get("sm_max_mhz") or peaks.get("sm_max_mhz")
     roofline = {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
                 "frac": fwd_tflops / peak, "traffic": recorded_traffic(w.name),
-                "kernel": "bsa_forward_kernel<128,128,128>",
-                "peak_source": f"{peak_src} bf16_tflops_sustained (dense bf16 cuBLAS, seconds-long loop)",
-                "fwd_ms": fwd_ms}
+                "kernel": f"bsa_forward_kernel<{w.d},{w.block},{w.block}>",
+                "peak_source": f"{peak_src} bf16_tflops (burst: dense bf16 cuBLAS, best of 10)",
+                "frac_sustained": fwd_tflops / peak_sus, "peak_sustained": peak_sus,
+                "frac_clock_normalised": (fwd_tflops / (peak * sm_mhz / sm_max)
+                                          if sm_mhz and sm_max else None),
+                "fwd_ms": fwd_ms_local}
 
     cpu = None
     parity = None
@@ -678,11 +797,11 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) bf16 q/k/v, PSA-style stripe masks)",
-            "config": workload_config(w, mask), "roofline": roofline, "cpu_baseline": cpu,
-            "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
-            "clocks": sampler.summary(t_wall0, t_wall1),
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": f"synthetic (seeded N(0,1) bf16 q/k/v, {w.mask_kind} masks)",
+            "config": workload_config(w_all, mask_all, world), "roofline": roofline,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
             "peak_frac_step": value / peak,
             "parity": parity,
             "next_rows": next_rows,

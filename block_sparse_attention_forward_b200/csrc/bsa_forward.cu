@@ -117,16 +117,20 @@ struct Barriers {
 };
 
 // Bounded wait, slow path: spin until the phase of `parity` completed (true)
-// or this CTA gives up (timeout here, or another role already aborted).
+// or this CTA gives up (timeout here, or another role already aborted).  With
+// abort == nullptr the wait ignores the other roles and ends only on the
+// phase or the timeout: the drains use it, so that a CTA that is giving up
+// still lets its copies land and its products finish before it frees TMEM
+// and exits.
 __device__ __noinline__ bool wait_barrier_slow(uint32_t bar, uint32_t parity, volatile int* abort,
                                                uint64_t timeout_ns = kTimeoutNs) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
-      if (*abort) return false;
+      if (abort && *abort) return false;
       if (global_timer_ns() - t0 > timeout_ns) {
-        *abort = 1;
+        if (abort) *abort = 1;
         atomicExch(&g_bsa_device_error, int(BSA_ERR_TIMEOUT));
         return false;
       }
@@ -309,10 +313,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) {
-        // let the copies already issued land before the CTA exits
+        // let the copies already issued land before the CTA exits (the wait
+        // ignores the abort flag, which is set by now)
         const uint32_t first = item > C::kStages ? item - C::kStages : 0;
         for (uint32_t i = first; i < item; ++i)
-          wait_barrier(smem_addr(&bars->kv_full[i % C::kStages]), (i / C::kStages) & 1, abort);
+          wait_barrier_slow(smem_addr(&bars->kv_full[i % C::kStages]), (i / C::kStages) & 1,
+                            nullptr);
       }
     }
   } else if (warp == 5) {
@@ -399,8 +405,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         g += cnt;
       }
       // drain: every MMA issued by this thread completes before TMEM is freed
+      // (the wait ignores the abort flag: only the phase or the timeout ends it)
       mma_commit(smem_addr(&bars->drain));
-      wait_fast(smem_addr(&bars->drain), 0, abort);
+      wait_barrier_slow(smem_addr(&bars->drain), 0, nullptr);
     }
   } else {
     // ------------------------------------------------------------ softmax (warps 0-3)

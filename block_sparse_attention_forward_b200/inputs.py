@@ -17,8 +17,11 @@ Block coordinates used by the mask generators.  The blocks index the
 tile-major (permuted) token order, where ragged edge tiles are concatenated,
 so a block is not always one tile.  The generators therefore give block i the
 coordinate (slab, spatial) with slab = floor(i * n_slabs / nb) (n_slabs =
-ceil(T / tile_t)) and spatial = i - (first block of that slab).  This only
-shapes the synthetic masks; the kernels treat every mask alike.
+ceil(T / tile_t)) and spatial = i - (first block of that slab).  The top-p
+generator pools q and k over each block's tokens; its grid is a whole number
+of block-sized tiles, so a reshape groups the frame-major tokens into those
+tiles.  This only shapes the synthetic masks (both the kernels and the oracle
+consume the same mask); the kernels treat every mask alike.
 """
 from __future__ import annotations
 
@@ -190,23 +193,31 @@ def _mask_psa_stripes(w: Workload, rng: np.random.Generator) -> np.ndarray:
     return best
 
 
+def _tile_means(x: torch.Tensor, w: Workload) -> torch.Tensor:
+    """Mean of each 3-D tile of a frame-major [T*Hs*Ws, d] tensor, tiles in
+    (tile_t, tile_y, tile_x) row-major order: [nb, d] fp64.  Only for grids the
+    tile divides, with one tile per block (a reshape groups the tokens)."""
+    t = x.double().view(w.T // w.tt, w.tt, w.Hs // w.th, w.th, w.Ws // w.tw, w.tw, w.d)
+    return t.mean(dim=(1, 3, 5)).reshape(-1, w.d)
+
+
 def _mask_top_p(w: Workload, rng: np.random.Generator, q: torch.Tensor, k: torch.Tensor,
                 p: float = 0.9) -> np.ndarray:
     """Top-p block masks from mean-pooled q/k block scores, temperature per head
     found by bisection so that the head's sparsity hits a target ~ U[0.80, 0.95].
 
-    Pooling runs over consecutive chunks of `block` frame-major tokens.
+    Pooling runs over the tokens of each attention block, that is over each
+    3-D tile of the token grid (the blocks the kernels walk); the grid must be
+    a whole number of tiles of `block` tokens each.
     """
+    if (w.T % w.tt or w.Hs % w.th or w.Ws % w.tw or w.tt * w.th * w.tw != w.block):
+        raise ValueError("top-p masks need a grid of whole tiles of one block each")
     m = np.zeros((w.B, w.H, w.nb, w.nb), dtype=np.uint8)
-    nb, blk = w.nb, w.block
+    nb = w.nb
     for b in range(w.B):
         for h in range(w.H):
-            qh = torch.zeros(w.n_pad, w.d)
-            kh = torch.zeros(w.n_pad, w.d)
-            qh[: w.n] = q[b, h].float()
-            kh[: w.n] = k[b, h].float()
-            qbar = qh.view(nb, blk, w.d).mean(1).double()
-            kbar = kh.view(nb, blk, w.d).mean(1).double()
+            qbar = _tile_means(q[b, h], w)
+            kbar = _tile_means(k[b, h], w)
             raw = (qbar @ kbar.T) / math.sqrt(w.d)
             target = rng.uniform(0.80, 0.95)
 

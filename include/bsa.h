@@ -122,10 +122,13 @@ bsa_status bsa_pack_mask(const uint8_t* dense, int B, int H, int nb_q, int nb_k,
  * 40 heads of 1024 query blocks of 1024 key blocks, B = 1, fits); a larger
  * call returns BSA_ERR_WORKSPACE (use bsa_pack_mask).  The first call on each device
  * looks up the array's device address (cudaGetSymbolAddress) with that device
- * current, so make that first call before any stream capture.  All calls share
- * the one array: calls whose kernels overlap on a GPU (for example on two
- * streams at once) race and give wrong results; calls in order on one stream
- * are safe, since each call clears the scratch it uses.  Other errors as for
+ * current, so make that first call before any stream capture; the address is
+ * kept for the life of the process, so a device reset (cudaDeviceReset) or a
+ * driver context other than the device's primary one is not supported.  All
+ * calls share the one array, which keeps the last call's contents: calls whose
+ * kernels overlap on a GPU (for example on two streams at once) race and give
+ * wrong results; calls in order on one stream are safe, since each call writes
+ * every scratch entry it reads before reading it.  Other errors as for
  * bsa_pack_mask; BSA_ERR_LAUNCH also if the address lookup fails.
  * ------------------------------------------------------------------------- */
 bsa_status bsa_pack_mask_noalloc(const uint8_t* dense, int B, int H, int nb_q, int nb_k,

@@ -79,7 +79,7 @@ def _load():
             lib.oracle_pack_bits.argtypes = [P, I64, I, P]
             lib.oracle_crm_lists.argtypes = [P, I64, I, P, P, P]
             lib.oracle_crm_lists.restype = I64
-            lib.oracle_schedule.argtypes = [P, I64, I64, P]
+            lib.oracle_schedule.argtypes = [P, I64, P]
             lib.oracle_tile_order.argtypes = [I, I, I, I, I, I, P]
             lib.oracle_permute.argtypes = [P, P, I64, I64, I64, I, P]
             lib.oracle_unpermute.argtypes = [P, P, I64, I64, I64, I, P]
@@ -138,13 +138,12 @@ def crm_lists(bits: np.ndarray):
     return counts, offsets, col_idx[:total]
 
 
-def schedule(counts: np.ndarray, nb_q: int = 0) -> np.ndarray:
-    """Work order of the rows: by count, largest first, stable; with nb_q > 0
-    (rows per head) the head-major form when the count order mixes more than 8
-    heads per window of 148 entries (see oracle.c)."""
+def schedule(counts: np.ndarray) -> np.ndarray:
+    """Work order of the rows: by kept-block count, largest first, ties by
+    ascending row id (a stable sort)."""
     counts = np.ascontiguousarray(counts, dtype=np.int32)
     out = np.zeros(counts.size, dtype=np.int32)
-    _load().oracle_schedule(_ptr(counts), counts.size, int(nb_q), _ptr(out))
+    _load().oracle_schedule(_ptr(counts), counts.size, _ptr(out))
     return out
 
 

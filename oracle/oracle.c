@@ -149,16 +149,12 @@ int64_t oracle_crm_lists(const uint32_t* bits, int64_t rows, int n_words, int32_
 }
 
 /* Schedule: row ids ordered by kept-block count, largest first; rows with
- * equal counts keep ascending row order.  Written as the plainest counting
- * order: for each count value from the largest down, list its rows.
- *
- * The pages are silent on the work order; this is the library's stated rule.
- * When nb_q > 0, rows belong to heads h = r / nb_q.  Over the count order's
- * full windows of 148 consecutive entries, the distinct heads of each window
- * are counted.  If their total exceeds 8 per window (and there are at most
- * 8192 heads and 8192 rows per head), the schedule becomes: heads in
- * ascending order, inside each head the same counting order. */
-void oracle_schedule(const int32_t* counts, int64_t rows, int64_t nb_q, int32_t* schedule) {
+ * equal counts keep ascending row order (a stable sort).  Written as the
+ * plainest counting order: for each count value from the largest down, list
+ * its rows.  The pages are silent on the work order; this is the order the
+ * load-balancing rule "most kept blocks first" names.  Any other work order
+ * gives the same attention output. */
+void oracle_schedule(const int32_t* counts, int64_t rows, int32_t* schedule) {
   int32_t max_count = 0;
   for (int64_t r = 0; r < rows; ++r)
     if (counts[r] > max_count) max_count = counts[r];
@@ -166,26 +162,6 @@ void oracle_schedule(const int32_t* counts, int64_t rows, int64_t nb_q, int32_t*
   for (int32_t c = max_count; c >= 0; --c)
     for (int64_t r = 0; r < rows; ++r)
       if (counts[r] == c) schedule[pos++] = (int32_t)r;
-
-  if (nb_q <= 0) return;
-  const int64_t heads = rows / nb_q, windows = rows / 148;
-  if (windows == 0 || heads > 8192 || nb_q > 8192) return;
-  int64_t distinct_total = 0;
-  for (int64_t w = 0; w < windows; ++w) {
-    for (int64_t i = 0; i < 148; ++i) {
-      const int64_t h = schedule[w * 148 + i] / nb_q;
-      int seen_before = 0;
-      for (int64_t k = 0; k < i; ++k)
-        if (schedule[w * 148 + k] / nb_q == h) seen_before = 1;
-      if (!seen_before) ++distinct_total;
-    }
-  }
-  if (distinct_total <= 8 * windows) return;
-  pos = 0;
-  for (int64_t h = 0; h < heads; ++h)
-    for (int32_t c = max_count; c >= 0; --c)
-      for (int64_t r = h * nb_q; r < (h + 1) * nb_q; ++r)
-        if (counts[r] == c) schedule[pos++] = (int32_t)r;
 }
 
 /* ------------------------------------------------------------------ */

@@ -43,3 +43,58 @@ def compare_out(gpu_out: np.ndarray, ref_out: np.ndarray, gpu_lse: np.ndarray, r
     fin = ~neg_ref
     lse_err = float(np.max(np.abs(gpu_lse[fin].astype(np.float64) - ref_lse[fin]))) if fin.any() else 0.0
     return float(diff.max()) if diff.size else 0.0, float(diff.mean()) if diff.size else 0.0, lse_err
+
+
+# ---------------------------------------------------------------- schedule
+# Any work order gives the same attention output, so the schedule has several
+# correct values.  The oracle fixes one of them (count descending, ties by row
+# id); the library may instead take that order head by head.  A schedule is
+# valid when it is one of these two orders.  Which one the library picks is
+# its own policy, stated here (and in the pack kernels) and tested as such.
+
+def head_major_order(counts: np.ndarray, nb_q: int) -> np.ndarray:
+    """Heads ascending; inside a head, count descending, ties by row id."""
+    counts = np.asarray(counts).reshape(-1)
+    order = sorted(range(counts.size), key=lambda r: (r // nb_q, -int(counts[r]), r))
+    return np.array(order, dtype=np.int32)
+
+
+def schedule_form(sched: np.ndarray, counts: np.ndarray, nb_q: int) -> str:
+    """'count' or 'head' for a valid schedule; fails the test otherwise."""
+    import oracle
+    sched = np.asarray(sched).reshape(-1)
+    counts = np.asarray(counts).reshape(-1)
+    assert sched.size == counts.size
+    assert np.array_equal(np.sort(sched), np.arange(counts.size)), "not a permutation of the rows"
+    if np.array_equal(sched, oracle.schedule(counts)):
+        return "count"
+    assert np.array_equal(sched, head_major_order(counts, nb_q)), \
+        "neither the count order nor the count order taken per head"
+    return "head"
+
+
+POLICY_WINDOW = 148      # one wave of a B200: one tile per SM
+POLICY_MAX_HEADS = 8     # distinct heads per window, on average, above which it goes head-major
+POLICY_LIMIT = 8192      # heads and rows per head beyond which the check is skipped
+
+
+def policy_form(counts: np.ndarray, nb_q: int) -> str:
+    """The library's rule: over the count order's full windows of 148 entries,
+    count the distinct heads of each window; when they average more than 8 per
+    window, take the order head by head."""
+    import oracle
+    counts = np.asarray(counts, dtype=np.int32).reshape(-1)
+    heads = counts.size // nb_q
+    windows = counts.size // POLICY_WINDOW
+    if windows == 0 or heads > POLICY_LIMIT or nb_q > POLICY_LIMIT:
+        return "count"
+    order = oracle.schedule(counts)[: windows * POLICY_WINDOW].reshape(windows, POLICY_WINDOW)
+    distinct = sum(len(set((row // nb_q).tolist())) for row in order)
+    return "head" if distinct > POLICY_MAX_HEADS * windows else "count"
+
+
+def check_schedule(sched: np.ndarray, counts: np.ndarray, nb_q: int) -> str:
+    """Valid, and the form the library's policy picks."""
+    form = schedule_form(sched, counts, nb_q)
+    assert form == policy_form(counts, nb_q), (form, policy_form(counts, nb_q))
+    return form

@@ -186,3 +186,14 @@ def test_forward_rejects_bad_args(lib):
     bad = BsaMask(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 1, 2, 8, 8, 2)  # wrong words
     assert call(mask=bad) == 1
     assert call(out=P(0x10004)) == 3
+
+
+@pytest.mark.parametrize("B,H,nb_q,nb_k,expect", [(1, 1, 4096, 32766, 7),   # needs 131073 ints
+                                                  (1, 64, 4096, 600, 7),
+                                                  (1, 1, 1, 49152, 2)])     # past the packing cap
+def test_pack_noalloc_rejects_oversize_on_the_host(lib, B, H, nb_q, nb_k, expect):
+    # the built-in scratch holds 131072 ints; a call needing one more is
+    # refused before any CUDA call (the pointers are never used)
+    fake = ctypes.c_void_p(0x1000)
+    assert lib.bsa_pack_mask_noalloc(fake, B, H, nb_q, nb_k, fake, fake, fake, fake, fake,
+                                     None) == expect

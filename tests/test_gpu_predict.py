@@ -22,7 +22,7 @@ import torch
 
 import oracle
 from block_sparse_attention_forward_b200 import inputs as I
-from tests.helpers import bf16_bits
+from tests.helpers import bf16_bits, check_schedule
 
 pytestmark = pytest.mark.gpu
 
@@ -97,7 +97,7 @@ def _run(w, heads=None):
     np.testing.assert_array_equal(pm.row_offsets.cpu().numpy().astype(np.int64), offsets_ref)
     total = int(offsets_ref[-1])
     np.testing.assert_array_equal(pm.col_idx[:total].cpu().numpy(), cols_ref)
-    np.testing.assert_array_equal(pm.schedule.cpu().numpy(), oracle.schedule(counts_ref, pm.nb_q))
+    check_schedule(pm.schedule.cpu().numpy(), counts_ref, pm.nb_q)
     return equal, checked, gpu.mean()
 
 

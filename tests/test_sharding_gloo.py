@@ -70,3 +70,18 @@ def test_two_rank_head_sharding_matches_single_process(tmp_path):
     q, k, v, mask, n, block = _case()
     ref, _ = oracle.attention(q, k, v, mask, n, block)
     np.testing.assert_array_equal(gathered, ref)
+
+
+@pytest.mark.parametrize("name", ["tiny", "wan13b_480p", "wan14b_480p", "wan14b_720p",
+                                  "hunyuan_768p"])
+def test_rank_slices_cover_every_head_once(name):
+    # bench.py --gpus N splits one problem by flat head index: for each
+    # workload shape and N in 1..8 the ranks' slices cover every (b, h) once
+    from block_sparse_attention_forward_b200 import inputs as I
+    w = I.WORKLOADS[name]
+    for world in range(1, 9):
+        seen = np.zeros(w.B * w.H, dtype=np.int64)
+        for rank in range(world):
+            lo, hi = head_range(w.B * w.H, world, rank)
+            seen[lo:hi] += 1
+        assert np.all(seen == 1), (name, world)
