@@ -574,9 +574,13 @@ def shard_workload(w, q, k, v, mask, world: int, rank: int):
 
     from block_sparse_attention_forward_b200.sharding import head_range
     lo, hi = head_range(w.B * w.H, world, rank)
-    flat = lambda x: x.reshape(1, w.B * w.H, *x.shape[2:])[:, lo:hi].contiguous()  # noqa: E731
+
+    def flat(x):
+        y = x.reshape(1, w.B * w.H, *x.shape[2:])[:, lo:hi]
+        return np.ascontiguousarray(y) if isinstance(y, np.ndarray) else y.contiguous()
+
     ws = dataclasses.replace(w, B=1, H=hi - lo)
-    return ws, flat(q), flat(k), flat(v), np.ascontiguousarray(flat(mask)), (lo, hi)
+    return ws, flat(q), flat(k), flat(v), flat(mask), (lo, hi)
 
 
 def main():
