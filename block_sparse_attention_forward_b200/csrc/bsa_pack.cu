@@ -23,9 +23,10 @@
 //                   tile's warps take turns placing their rows at their
 //                   count's next slot -- in row order, so the sort is stable.
 //   5. head_mix:    distinct heads per window of 148 entries of that order.
-//   6. head_major:  if they exceed 8 per window on average, the schedule
-//                   becomes count-descending within each head, heads in order
-//                   (a counting sort per head, one CTA each).
+//   6. head_major:  if those heads' K and V, on average over the windows, do
+//                   not fit in L2, the schedule becomes count-descending
+//                   within each head, heads in order (a counting sort per
+//                   head, one CTA each).
 //   7. write_lists: one warp per row; words are taken one at a time and each
 //                   lane writes its key block at the row's running offset, so
 //                   each store instruction writes consecutive addresses.
@@ -312,11 +313,14 @@ __global__ void __launch_bounds__(kTileRows)
 // HunyuanVideo 768p: 20 of 24 heads per wave of 148 tiles, 139 GB of DRAM
 // reads per forward).  So the mean number of distinct heads over the order's
 // full windows of kMixWindow entries (one wave of a B200) is measured, and
-// when it exceeds kMixHeads the schedule becomes count-descending within each
-// head, heads in order (ties by row id, as above).
+// when that many heads' K and V -- nb_k key blocks of kKeyBlockBytes each --
+// exceed the L2 capacity, the schedule becomes count-descending within each
+// head, heads in order (ties by row id, as above).  The packing does not see
+// the head dimension or the block size, so a key block is costed as 128
+// tokens of K and V at d = 128 in bf16.
 // ---------------------------------------------------------------------------
 constexpr int kMixWindow = 148;
-constexpr int kMixHeads = 8;
+constexpr int64_t kKeyBlockBytes = 2 * 128 * 128 * 2;
 constexpr int kMixMaxHeads = 8192;    // bitmap of one window: 1 KB of shared memory per warp
 constexpr int kMixMaxRowsPerHead = 8192;
 constexpr int kMixWarps = 8;
@@ -345,8 +349,8 @@ __global__ void __launch_bounds__(kMixWarps * 32)
   if (lane == 0) atomicAdd(mix_sum, distinct);
 }
 
-// One CTA per head (kTileRows threads), only when the windows mixed more than
-// kMixHeads heads on average: a counting sort of the head's rows by count,
+// One CTA per head (kTileRows threads), only when the windows' heads, on
+// average, do not fit in L2 together: a counting sort of the head's rows by count,
 // descending.  Histogram of keys d = nb_k - count in shared memory, exclusive
 // scan of it (chunks of kTileRows bins), then the rows in order, a chunk of
 // kTileRows at a time, the chunk's warps taking turns: each lane's slot is
@@ -354,8 +358,10 @@ __global__ void __launch_bounds__(kMixWarps * 32)
 // counts keep ascending row order.
 __global__ void __launch_bounds__(kTileRows)
     head_major_kernel(const int32_t* __restrict__ counts, int nb_q, int nb_k, int windows,
-                      const int32_t* __restrict__ mix_sum, int32_t* __restrict__ schedule) {
-  if (*mix_sum <= kMixHeads * windows) return;  // the count order keeps few heads per wave
+                      int64_t l2_bytes, const int32_t* __restrict__ mix_sum,
+                      int32_t* __restrict__ schedule) {
+  // the count order's waves touch few enough heads: their K and V stay in L2
+  if (int64_t(*mix_sum) * nb_k * kKeyBlockBytes <= int64_t(windows) * l2_bytes) return;
   extern __shared__ int32_t next_slot[];        // nb_k + 1 bins
   __shared__ int scan_smem[33];
   const int bins = nb_k + 1;
@@ -501,8 +507,12 @@ bsa_status launch_offsets_schedule_lists(const uint32_t* bits, const int32_t* co
     if (cudaFuncSetAttribute(head_major_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(bins_bytes)) != cudaSuccess)
       return BSA_ERR_LAUNCH;
-    head_major_kernel<<<heads, kTileRows, bins_bytes, s>>>(counts, nb_q, nb_k, windows, mix_sum,
-                                                          schedule);
+    int dev = 0, l2 = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 <= 0)
+      return BSA_ERR_LAUNCH;
+    head_major_kernel<<<heads, kTileRows, bins_bytes, s>>>(counts, nb_q, nb_k, windows,
+                                                          int64_t(l2), mix_sum, schedule);
     if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
   }
   if (col_idx) {

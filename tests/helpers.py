@@ -74,14 +74,20 @@ def schedule_form(sched: np.ndarray, counts: np.ndarray, nb_q: int) -> str:
 
 
 POLICY_WINDOW = 148      # one wave of a B200: one tile per SM
-POLICY_MAX_HEADS = 8     # distinct heads per window, on average, above which it goes head-major
+POLICY_KEY_BLOCK_BYTES = 2 * 128 * 128 * 2  # K and V of a 128-token key block, d = 128, bf16
 POLICY_LIMIT = 8192      # heads and rows per head beyond which the check is skipped
 
 
-def policy_form(counts: np.ndarray, nb_q: int) -> str:
+def device_l2_bytes() -> int:
+    import torch
+    return int(torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size)
+
+
+def policy_form(counts: np.ndarray, nb_q: int, nb_k: int, l2_bytes: int) -> str:
     """The library's rule: over the count order's full windows of 148 entries,
-    count the distinct heads of each window; when they average more than 8 per
-    window, take the order head by head."""
+    count the distinct heads of each window; when that many heads' K and V
+    (nb_k key blocks each) exceed the L2 capacity on average, take the order
+    head by head."""
     import oracle
     counts = np.asarray(counts, dtype=np.int32).reshape(-1)
     heads = counts.size // nb_q
@@ -90,11 +96,15 @@ def policy_form(counts: np.ndarray, nb_q: int) -> str:
         return "count"
     order = oracle.schedule(counts)[: windows * POLICY_WINDOW].reshape(windows, POLICY_WINDOW)
     distinct = sum(len(set((row // nb_q).tolist())) for row in order)
-    return "head" if distinct > POLICY_MAX_HEADS * windows else "count"
+    return ("head" if distinct * nb_k * POLICY_KEY_BLOCK_BYTES > windows * l2_bytes
+            else "count")
 
 
-def check_schedule(sched: np.ndarray, counts: np.ndarray, nb_q: int) -> str:
-    """Valid, and the form the library's policy picks."""
+def check_schedule(sched: np.ndarray, counts: np.ndarray, nb_q: int, nb_k: int,
+                   l2_bytes: int | None = None) -> str:
+    """Valid, and the form the library's policy picks (L2 size of the current
+    device unless given)."""
     form = schedule_form(sched, counts, nb_q)
-    assert form == policy_form(counts, nb_q), (form, policy_form(counts, nb_q))
+    l2 = device_l2_bytes() if l2_bytes is None else l2_bytes
+    assert form == policy_form(counts, nb_q, nb_k, l2), (form, policy_form(counts, nb_q, nb_k, l2))
     return form

@@ -28,7 +28,7 @@ def _pack_and_compare(dense: np.ndarray):
     np.testing.assert_array_equal(pm.row_offsets.cpu().numpy().astype(np.int64), offsets_ref)
     total = int(offsets_ref[-1])
     np.testing.assert_array_equal(pm.col_idx[:total].cpu().numpy(), col_ref)
-    return check_schedule(pm.schedule.cpu().numpy(), counts_ref, nbq)
+    return check_schedule(pm.schedule.cpu().numpy(), counts_ref, nbq, nbk)
 
 
 @pytest.mark.parametrize("name", ["tiny", "wan13b_480p", "wan14b_480p", "wan14b_720p",
@@ -68,7 +68,8 @@ def test_pack_schedule_head_major_long_heads_and_batches(cuda_ok):
 
 
 def test_pack_schedule_stays_count_order_when_heads_separate(cuda_ok):
-    # disjoint count ranges per head: few heads per window, the count order stays
+    # disjoint count ranges per head: about two heads per window, whose K and V
+    # fit in L2, so the count order stays
     rng = np.random.default_rng(7)
     counts = np.stack([h * 20 + rng.integers(0, 15, size=96) for h in range(12)])
     dense = _mask_with_counts(counts, 256, 15)
@@ -78,11 +79,15 @@ def test_pack_schedule_stays_count_order_when_heads_separate(cuda_ok):
 @pytest.mark.parametrize("heads,form", [(8, "count"), (9, "head")])
 def test_pack_schedule_mix_threshold(cuda_ok, heads, form):
     # row i of every head keeps 200 - i blocks: each count level lists all the
-    # heads, so every window of 148 holds all of them; 8 heads per window stays
-    # in count order, 9 is more than 8 and turns head-major
+    # heads, so every window of 148 holds all of them; nb_k is chosen so that
+    # this GPU's L2 holds the K and V of 8.5 heads: 8 heads per window stay in
+    # count order, 9 turn head-major
+    from tests.helpers import POLICY_KEY_BLOCK_BYTES, device_l2_bytes
     nbq = 148
+    nbk = int(device_l2_bytes() / (8.5 * POLICY_KEY_BLOCK_BYTES))
+    assert nbk >= 200
     counts = np.tile(200 - np.arange(nbq), (heads, 1))
-    dense = _mask_with_counts(counts, 256, 13)
+    dense = _mask_with_counts(counts, nbk, 13)
     assert _pack_and_compare(dense) == form
 
 

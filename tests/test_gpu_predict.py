@@ -97,7 +97,7 @@ def _run(w, heads=None):
     np.testing.assert_array_equal(pm.row_offsets.cpu().numpy().astype(np.int64), offsets_ref)
     total = int(offsets_ref[-1])
     np.testing.assert_array_equal(pm.col_idx[:total].cpu().numpy(), cols_ref)
-    check_schedule(pm.schedule.cpu().numpy(), counts_ref, pm.nb_q)
+    check_schedule(pm.schedule.cpu().numpy(), counts_ref, pm.nb_q, pm.nb_k)
     return equal, checked, gpu.mean()
 
 

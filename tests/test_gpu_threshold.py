@@ -24,17 +24,17 @@ pytestmark = pytest.mark.gpu
 def _oracle_pack(dense):
     bits = oracle.pack_bits(dense)
     counts, offsets, cols = oracle.crm_lists(bits)
-    return bits, counts, offsets, cols, dense.shape[2]
+    return bits, counts, offsets, cols, dense.shape[2:]
 
 
 def _compare(pm, ref):
-    bits, counts, offsets, cols, nb_q = ref
+    bits, counts, offsets, cols, (nb_q, nb_k) = ref
     np.testing.assert_array_equal(pm.bits.cpu().numpy().view(np.uint32), bits)
     np.testing.assert_array_equal(pm.counts.cpu().numpy(), counts)
     np.testing.assert_array_equal(pm.row_offsets.cpu().numpy().astype(np.int64), offsets)
     total = int(offsets[-1])
     np.testing.assert_array_equal(pm.col_idx[:total].cpu().numpy(), cols)
-    check_schedule(pm.schedule.cpu().numpy(), counts, nb_q)
+    check_schedule(pm.schedule.cpu().numpy(), counts, nb_q, nb_k)
 
 
 def _pack_threshold_and_compare(thr, p, B=1):

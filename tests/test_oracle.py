@@ -103,15 +103,17 @@ def test_schedule_ties_keep_row_order_and_all_rows_appear():
 def test_library_schedule_policy_boundary(heads, form):
     # the library's work-order policy (stated in tests/helpers.py, not part of
     # the oracle): row i of every head keeps 200 - i blocks, so each window of
-    # 148 count-order entries holds every head; 8 heads per window keeps the
-    # count order, 9 turns head-major
-    from tests.helpers import head_major_order, policy_form, schedule_form
-    nb_q = 148
+    # 148 count-order entries holds every head.  With L2 sized for 8.5 heads'
+    # K and V, 8 heads per window keep the count order and 9 turn head-major
+    from tests.helpers import (POLICY_KEY_BLOCK_BYTES, head_major_order, policy_form,
+                               schedule_form)
+    nb_q, nb_k = 148, 240
+    l2 = int(8.5 * nb_k * POLICY_KEY_BLOCK_BYTES)
     counts = np.tile(200 - np.arange(nb_q), heads).astype(np.int32)
-    assert policy_form(counts, nb_q) == form
+    assert policy_form(counts, nb_q, nb_k, l2) == form
     assert schedule_form(head_major_order(counts, nb_q), counts, nb_q) == "head"
     assert schedule_form(oracle.schedule(counts), counts, nb_q) == "count"
-    assert policy_form(counts[: 147], nb_q) == "count"  # no full window
+    assert policy_form(counts[: 147], nb_q, nb_k, l2) == "count"  # no full window
 
 def test_tile_order_divisible_matches_reshape():
     T, Hs, Ws, tt, th, tw = 4, 16, 16, 2, 8, 4

@@ -78,7 +78,7 @@ def _compare_with_oracle(got, m):
     np.testing.assert_array_equal(got["row_offsets"].cpu().numpy().astype(np.int64), offsets_ref)
     total = int(offsets_ref[-1])
     np.testing.assert_array_equal(got["col_idx"][:total].cpu().numpy(), col_ref)
-    check_schedule(got["schedule"].cpu().numpy(), counts_ref, m.shape[2])
+    check_schedule(got["schedule"].cpu().numpy(), counts_ref, m.shape[2], m.shape[3])
 
 
 def test_noalloc_pack_at_the_largest_size_that_fits(cuda_ok):
