@@ -556,6 +556,101 @@ def measure_by_length(dev, stream, peak_tflops: float, reuse=None):
     return {"by_length": rows, "by_length_peak": peak_tflops}
 
 
+def measure_power_loops(w, dev, seconds: float = 6.0):
+    """Power, SM clock and energy per FLOP of three kernels on the workload's
+    tensors, each looped for `seconds` while nvidia-smi samples every 100 ms: the
+    forward with the workload's mask, the forward with an all-ones mask, and
+    PyTorch's dense SDPA (context, not ours).  Under the 1 kW cap the clock settles
+    where the power meets the cap, so TFLOP/s per GHz and pJ per FLOP compare the
+    kernels' work per clock and per joule."""
+    import block_sparse_attention_forward_b200 as bsa
+    q, k, v = I.gen_qkv(w)
+    mask = I.gen_mask(w, q, k)
+    grid, tile = (w.T, w.Hs, w.Ws), (w.tt, w.th, w.tw)
+    qp, kp, vp = (bsa.tile_permute(t.to(dev), grid, tile, w.n_pad) for t in (q, k, v))
+    del q, k, v
+    pm = bsa.pack_mask(torch.from_numpy(mask).to(dev))
+    ones = bsa.pack_mask(torch.ones((w.B, w.H, w.nb, w.nb), dtype=torch.uint8, device=dev))
+    out = torch.empty_like(qp)
+    lse = torch.empty((w.B, w.H, w.n_pad), dtype=torch.float32, device=dev)
+    qd, kd, vd = (t[:, :, :w.n] for t in (qp, kp, vp))
+    tile_flop = 4.0 * w.d * w.block * w.block
+    cases = [
+        ("forward_mask", lambda: bsa.forward(qp, kp, vp, pm, w.n, w.block, out=out, lse=lse),
+         tile_flop * I.kept_tiles(mask)),
+        ("forward_all_ones", lambda: bsa.forward(qp, kp, vp, ones, w.n, w.block, out=out, lse=lse),
+         tile_flop * w.B * w.H * w.nb * w.nb),
+        ("torch_sdpa_dense", lambda: torch.nn.functional.scaled_dot_product_attention(qd, kd, vd),
+         4.0 * w.d * w.n * w.n * w.B * w.H),
+    ]
+    res = {}
+    stream = torch.cuda.current_stream(dev)
+    for name, fn, flops in cases:
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        sampler = PowerSampler(gpu_selector(dev))
+        sampler.start()
+        time.sleep(0.5)
+        t0 = time.time()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        n = 0
+        while time.time() - t0 < seconds:
+            fn()
+            n += 1
+            if n % 4 == 0:
+                torch.cuda.synchronize(dev)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        t1 = time.time()
+        sampler.stop()
+        ms = e0.elapsed_time(e1) / n
+        sm, watts, capped = sampler.summary(t0 + 0.5, t1)
+        tf = flops / (ms * 1e-3) / 1e12
+        res[name] = {"ms": ms, "tflops": tf, "sm_mhz": sm, "watts": watts,
+                     "pj_per_flop": (watts / (tf * 1e12) * 1e12) if watts else None,
+                     "tflops_per_ghz": (tf / sm * 1e3) if sm else None,
+                     "sw_power_cap_samples": capped, "calls": n}
+    if bsa.device_error() != 0:
+        raise RuntimeError("device error in the power loops")
+    return res
+
+
+class PowerSampler(ClockSampler):
+    """SM clock, power draw and the power-cap flag, sampled during a window."""
+
+    QUERY = "clocks.sm,power.draw,clocks_event_reasons.sw_power_cap"
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def summary(self, t0: float, t1: float):
+        sm, watts, capped = [], [], 0
+        for ts, line in self.lines:
+            if not (t0 <= ts <= t1):
+                continue
+            f = [x.strip() for x in line.split(",")]
+            try:
+                sm.append(float(f[0]))
+                watts.append(float(f[1]))
+                capped += f[2].lower().startswith("active")
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None, None, 0
+        return statistics.median(sm), statistics.median(watts), capped
+
+
 def workload_config(w, mask, world: int = 1):
     kept = I.kept_tiles(mask)
     total = w.B * w.H * w.nb * w.nb
@@ -598,6 +693,12 @@ def main():
                     help="measure only the threshold-map rows (a small case for profiling)")
     ap.add_argument("--no-by-length", action="store_true",
                     help="skip the forward / all-ones / SDPA comparison over the four workloads")
+    ap.add_argument("--power-loops", action="store_true",
+                    help="only loop the forward (mask, all-ones) and dense SDPA for a few seconds "
+                         "each and report power, SM clock and energy per FLOP")
+    ap.add_argument("--sdpa-only", action="store_true",
+                    help="only run dense SDPA three times on the workload's tensors (a small case "
+                         "for an ncu capture of its kernel)")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (smaller cases for profiling captures)")
     args = ap.parse_args()
@@ -615,6 +716,20 @@ def main():
     world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.power_loops:
+        res = measure_power_loops(w, dev)
+        if rank == 0:
+            print(json.dumps({"workload": w.name, "power_loops": res}), flush=True)
+        return 0
+    if args.sdpa_only:
+        g = torch.Generator().manual_seed(w.seed)
+        q, k, v = (torch.randn((w.B, w.H, w.n, w.d), generator=g).to(torch.bfloat16).to(dev)
+                   for _ in range(3))
+        for _ in range(3):
+            o = torch.nn.functional.scaled_dot_product_attention(q, k, v)
+        torch.cuda.synchronize(dev)
+        print(json.dumps({"workload": w.name, "sdpa_only": float(o.float().abs().mean())}))
+        return 0
     if args.only_next:
         peaks, _ = load_peaks()
         rows = measure_threshold_rows(w, dev, torch.cuda.current_stream(dev),
