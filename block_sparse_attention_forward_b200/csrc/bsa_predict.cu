@@ -17,11 +17,9 @@
 //   1. pool:        one CTA per (b, h, block); fp32 means of the block's
 //                   valid q and k rows into the workspace (HBM bound: q and k
 //                   are read once).
-//   2. score_topp:  one CTA per (b, h, 32 query blocks) when nb <= 1024
-//                   (score_topp_wide_kernel: 8 x 4 register tiles, key means
-//                   staged by cp.async two slices deep), else per 16 query
-//                   blocks (score_topp_kernel: 4 x 4 tiles).  Scores by fp32
-//                   FMA, in the same order of terms in both; then one warp per row: max, exp, sum, and the cut
+//   2. score_topp:  one CTA per (b, h, kRowsPerCta query blocks).  Scores by
+//                   fp32 FMA in 4 x 4 register tiles against key means staged
+//                   in shared memory; then one warp per row: max, exp, sum, and the cut
 //                   found by bisection on the bit patterns of the
 //                   (non-negative) exponentials -- the largest T with
 //                   sum(e_j >= T) >= top_p * sum(e) -- then ties at T taken
@@ -260,147 +258,6 @@ __global__ void __launch_bounds__(kScoreThreads)
                         counts + bh * nb + i0 + rr);
 }
 
-// Scores for up to kMaxBlocksWide key blocks: kRowsWide query blocks per CTA,
-// each thread an 8-row x 4-key register tile (rows 8 (t / 64) + a, keys
-// (t % 64) + 64 b of each pass of kKeyChunk keys), so that one 16-byte vector of
-// key means (a quarter warp's in distinct banks) feeds 8 FMA chains and one
-// broadcast vector of query means feeds 4: 12 vector loads per 128 FMAs.  The
-// key means are staged 32 dimensions at a time, two slices in flight
-// (cp.async into alternate buffers: the next slice's loads overlap this
-// slice's FMAs).  Then the same per-row cut as above.
-constexpr int kRowsWide = 32;
-constexpr int kMaxBlocksWide = 1024;
-constexpr int kSliceFloats = kKeyChunk * kKsStride;  // one staged slice of key means
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-template <int kPerLane>
-__global__ void __launch_bounds__(kScoreThreads)
-    score_topp_wide_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar, int H,
-                           int nb, int d, const float* __restrict__ tau,
-                           const float* __restrict__ top_p, uint32_t* __restrict__ bits,
-                           int32_t* __restrict__ counts) {
-  extern __shared__ float4 score_smem4[];
-  float* qs = reinterpret_cast<float*>(score_smem4);  // [kRowsWide][d]
-  float* ks = qs + kRowsWide * d;                     // [2][kKeyChunk][kKsStride]
-  float* sc = ks + 2 * kSliceFloats;                  // [kRowsWide][nb]
-  const int64_t bh = blockIdx.y;
-  const int h = int(bh % H);
-  const int i0 = blockIdx.x * kRowsWide;
-  const int rows = min(kRowsWide, nb - i0);
-  const float inv_denom = 1.0f / (sqrtf(float(d)) * __ldg(tau + h));
-  const int slices_per_chunk = d / kDSlice;
-  const int chunks = (nb + kKeyChunk - 1) / kKeyChunk;
-  const int n_slices = chunks * slices_per_chunk;
-
-  // slice s = (key chunk s / slices_per_chunk, dims 32 (s % slices_per_chunk))
-  // into buffer s & 1: 256 keys x 8 vectors, 8 per thread; keys past nb read
-  // zeros (source size 0)
-  auto stage = [&](int sl) {
-    const int j0 = (sl / slices_per_chunk) * kKeyChunk;
-    const int c0 = (sl % slices_per_chunk) * kDSlice;
-    float* buf = ks + (sl & 1) * kSliceFloats;
-    for (int e = threadIdx.x; e < kKeyChunk * (kDSlice / 4); e += kScoreThreads) {
-      const int key = e / (kDSlice / 4), part = e - key * (kDSlice / 4);
-      const bool in = j0 + key < nb;
-      const float* src = kbar + ((bh * nb + (in ? j0 + key : 0)) * d + c0 + part * 4);
-      cp_async16(static_cast<uint32_t>(__cvta_generic_to_shared(buf + key * kKsStride + part * 4)),
-                 src, in ? 16u : 0u);
-    }
-    cp_async_commit();
-  };
-
-  stage(0);
-  for (int e = threadIdx.x; e < kRowsWide * d; e += kScoreThreads) {
-    const int r = e / d, c = e - r * d;
-    qs[e] = r < rows ? qbar[(bh * nb + i0 + r) * d + c] : 0.0f;
-  }
-  const int rg = threadIdx.x / 64, kg = threadIdx.x % 64;
-  float acc[8][4];
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-  for (int sl = 0; sl < n_slices; ++sl) {
-    if (sl + 1 < n_slices) {
-      stage(sl + 1);
-      cp_async_wait<1>();  // this slice has landed (the next may be in flight)
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const int c0 = (sl % slices_per_chunk) * kDSlice;
-    const float* buf = ks + (sl & 1) * kSliceFloats;
-#pragma unroll
-    for (int c4 = 0; c4 < kDSlice / 4; ++c4) {
-      float4 qv[8], kv[4];
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-        qv[a] = *reinterpret_cast<const float4*>(qs + (rg * 8 + a) * d + c0 + c4 * 4);
-#pragma unroll
-      for (int b = 0; b < 4; ++b)
-        kv[b] = *reinterpret_cast<const float4*>(buf + (kg + 64 * b) * kKsStride + c4 * 4);
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          acc[a][b] = fmaf(qv[a].x, kv[b].x, acc[a][b]);
-          acc[a][b] = fmaf(qv[a].y, kv[b].y, acc[a][b]);
-          acc[a][b] = fmaf(qv[a].z, kv[b].z, acc[a][b]);
-          acc[a][b] = fmaf(qv[a].w, kv[b].w, acc[a][b]);
-        }
-    }
-    if (sl % slices_per_chunk == slices_per_chunk - 1) {  // a key chunk is complete
-      const int j0 = (sl / slices_per_chunk) * kKeyChunk;
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int key = j0 + kg + 64 * b;
-          if (key < nb) sc[(rg * 8 + a) * nb + key] = acc[a][b] * inv_denom;
-          acc[a][b] = 0.0f;
-        }
-    }
-    __syncthreads();  // every thread is done with this buffer before it is refilled
-  }
-
-  const int warp = threadIdx.x >> 5;
-  const float p_h = __ldg(top_p + h);
-  for (int rr = warp; rr < rows; rr += kScoreThreads / 32)
-    top_p_row<kPerLane>(sc + rr * nb, nb, p_h, bits + (bh * nb + i0 + rr) * ((nb + 31) / 32),
-                        counts + bh * nb + i0 + rr);
-}
-
-size_t score_wide_smem_bytes(int nb, int d) {
-  return sizeof(float) * (size_t(kRowsWide) * d + 2 * size_t(kSliceFloats) +
-                          size_t(kRowsWide) * nb);
-}
-
-template <int kPerLane>
-bsa_status launch_score_wide(int nb, int d, int64_t BH, cudaStream_t s, const float* qbar,
-                             const float* kbar, int H, const float* tau, const float* top_p,
-                             uint32_t* bits, int32_t* counts) {
-  const size_t smem = score_wide_smem_bytes(nb, d);
-  if (cudaFuncSetAttribute(score_topp_wide_kernel<kPerLane>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-    return BSA_ERR_LAUNCH;
-  const dim3 grid(unsigned((nb + kRowsWide - 1) / kRowsWide), unsigned(BH));
-  score_topp_wide_kernel<kPerLane><<<grid, kScoreThreads, smem, s>>>(qbar, kbar, H, nb, d, tau,
-                                                                     top_p, bits, counts);
-  return bsa::launch_status() == BSA_OK ? BSA_OK : BSA_ERR_LAUNCH;
-}
-
 size_t score_smem_bytes(int nb, int d) {
   return sizeof(float) * (size_t(kRowsPerCta) * d + size_t(kKeyChunk) * kKsStride +
                           size_t(kRowsPerCta) * nb);
@@ -473,16 +330,7 @@ extern "C" bsa_status bsa_predict_top_p(const void* q, const void* k, int B, int
   const dim3 grid(unsigned((nb + kRowsPerCta - 1) / kRowsPerCta), unsigned(BH));
   const int per_lane = (nb + 31) / 32;
   bsa_status st;
-  if (nb <= kMaxBlocksWide) {
-    if (per_lane <= 8)
-      st = launch_score_wide<8>(nb, d, BH, s, qbar, kbar, H, tau, top_p, bits, counts);
-    else if (per_lane <= 16)
-      st = launch_score_wide<16>(nb, d, BH, s, qbar, kbar, H, tau, top_p, bits, counts);
-    else if (per_lane <= 20)
-      st = launch_score_wide<20>(nb, d, BH, s, qbar, kbar, H, tau, top_p, bits, counts);
-    else
-      st = launch_score_wide<32>(nb, d, BH, s, qbar, kbar, H, tau, top_p, bits, counts);
-  } else if (per_lane <= 8)
+  if (per_lane <= 8)
     st = launch_score<8>(grid, smem, s, qbar, kbar, H, nb, d, tau, top_p, bits, counts);
   else if (per_lane <= 16)
     st = launch_score<16>(grid, smem, s, qbar, kbar, H, nb, d, tau, top_p, bits, counts);
