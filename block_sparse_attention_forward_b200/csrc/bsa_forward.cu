@@ -70,6 +70,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256, kTmemQ = 384;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
+constexpr int kMaxListRounds = 2048;  // tiles per CTA for tiles of several query blocks
 
 struct FwdParams {
   const __nv_bfloat16* q;   // [BH, n_pad, d]
@@ -79,6 +80,7 @@ struct FwdParams {
   float* lse;               // [BH, n_pad]
   int BH, nb_q, nb_k, words, n_valid, n_pad;
   int num_tiles, tiles_per_head;
+  int use_list;  // tiles of several query blocks: taken in schedule order via a per-CTA list
   float scale_log2;
 };
 
@@ -91,13 +93,17 @@ struct Cfg {
   static constexpr uint32_t kKVRegion = kTileN * 128;
   static constexpr uint32_t kSlotBytes = kRegions * kKVRegion;  // one K or V tile
   static constexpr uint32_t kMaxSmem = 227u * 1024u;
-  static constexpr int kFitStages = int((kMaxSmem - 256 - 1024) / kSlotBytes);
+  // tiles of several query blocks keep this CTA's list of tiles in shared memory
+  static constexpr int kListInts = R > 1 ? kMaxListRounds : 0;
+  static constexpr uint32_t kListBytes = 4u * kListInts + (R > 1 ? 64u : 0u);
+  static constexpr int kFitStages = int((kMaxSmem - 256 - kListBytes - 1024) / kSlotBytes);
   static constexpr int kStages = kFitStages > kMaxStages ? kMaxStages : kFitStages;
   static constexpr uint32_t kOffKV = 0;
   static constexpr uint32_t kOffBar = kOffKV + kStages * kSlotBytes;
-  // + barriers + alignment slack; at least 120 KB so that a second CTA never
-  // fits on the SM (each CTA owns all 512 TMEM columns)
-  static constexpr uint32_t kSmemUsed = kOffBar + 256 + 1024;
+  static constexpr uint32_t kOffList = kOffBar + 256;
+  // + barriers + list + alignment slack; at least 120 KB so that a second CTA
+  // never fits on the SM (each CTA owns all 512 TMEM columns)
+  static constexpr uint32_t kSmemUsed = kOffList + kListBytes + 1024;
   static constexpr uint32_t kSmemBytes = kSmemUsed > 120u * 1024u ? kSmemUsed : 120u * 1024u;
   static constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false);
   static_assert(kSmemUsed <= kMaxSmem, "shared memory budget");
@@ -200,20 +206,87 @@ struct TileInfo {
   const uint32_t* row1;  // second query block's CRM row (two blocks per tile), or null
 };
 
+// The tile of round r for this CTA, as the flat row of its first query block;
+// false when the CTA has no tile in this round.  One query block per tile:
+// schedule position snake_tile(r).  Several: entry r of the CTA's list (the
+// tiles in schedule order of their first row, dealt the same way), or, when
+// the list does not fit, the tiles in head order.
 template <int R>
-__device__ __forceinline__ TileInfo tile_info(const FwdParams& p, int tile) {
-  TileInfo t;
-  if (R == 1) {
-    const int row = __ldg(p.schedule + tile);
-    t.bh = row / p.nb_q;
-    t.qb0 = row - t.bh * p.nb_q;
-  } else {
-    t.bh = tile / p.tiles_per_head;
-    t.qb0 = (tile - t.bh * p.tiles_per_head) * R;
+__device__ __forceinline__ bool round_tile(const FwdParams& p, const int32_t* list, int r,
+                                           int& row) {
+  if (R > 1 && p.use_list) {
+    row = list[r];
+    return row >= 0;
   }
-  t.row0 = p.bits + (int64_t(t.bh) * p.nb_q + t.qb0) * p.words;
+  const int tile = snake_tile(r);
+  if (tile >= p.num_tiles) return false;
+  if (R == 1) {
+    row = __ldg(p.schedule + tile);
+  } else {
+    const int bh = tile / p.tiles_per_head;
+    row = bh * p.nb_q + (tile - bh * p.tiles_per_head) * R;
+  }
+  return true;
+}
+
+template <int R>
+__device__ __forceinline__ TileInfo tile_info(const FwdParams& p, int row) {
+  TileInfo t;
+  t.bh = row / p.nb_q;
+  t.qb0 = row - t.bh * p.nb_q;
+  t.row0 = p.bits + int64_t(row) * p.words;
   t.row1 = (R > 1 && t.qb0 + 1 < p.nb_q) ? t.row0 + p.words : nullptr;
   return t;
+}
+
+// Builds this CTA's list of tiles of R query blocks (all threads of the block
+// take part): the rows whose query block starts a tile (qb % R == 0) in
+// schedule order get ranks k = 0, 1, ...; rank k goes to round k / G, at index
+// k % G of an even round and G - 1 - (k % G) of an odd one (as snake_tile).
+template <int R>
+__device__ void build_tile_list(const FwdParams& p, int32_t* list, int32_t* scan, int n_rounds) {
+  const int G = int(gridDim.x), warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kWarps = kThreads / 32;
+  for (int r = threadIdx.x; r < n_rounds; r += kThreads) list[r] = -1;
+  const int rows = p.BH * p.nb_q;
+  int base = 0;
+  for (int c0 = 0; c0 < rows; c0 += kThreads * 8) {
+    int vals[8];
+    int cnt = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = c0 + int(threadIdx.x) * 8 + e;
+      const int row = i < rows ? __ldg(p.schedule + i) : -1;
+      const bool first = row >= 0 && (row % p.nb_q) % R == 0;
+      vals[e] = first ? row : -1;
+      cnt += first ? 1 : 0;
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    __syncthreads();  // the previous chunk's reads of scan[] are done
+    if (lane == 31) scan[warp] = incl;
+    __syncthreads();
+    int wbase = 0, total = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      const int x = scan[w];
+      wbase += w < warp ? x : 0;
+      total += x;
+    }
+    int k = base + wbase + incl - cnt;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (vals[e] < 0) continue;
+      const int round = k / G, idx = k - round * G;
+      const int owner = (round & 1) ? G - 1 - idx : idx;
+      if (owner == int(blockIdx.x) && round < n_rounds) list[round] = vals[e];
+      ++k;
+    }
+    base += total;
+  }
 }
 
 __device__ __forceinline__ int union_count(const TileInfo& t, int words) {
@@ -233,9 +306,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   Barriers* bars = reinterpret_cast<Barriers*>(smem + C::kOffBar);
+  int32_t* list = reinterpret_cast<int32_t*>(smem + C::kOffList);
   const uint32_t sKV = smem_addr(smem + C::kOffKV);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &bars->abort;
+  const int n_rounds = (p.num_tiles + int(gridDim.x) - 1) / int(gridDim.x);
+  if constexpr (C::R > 1) {
+    if (p.use_list) build_tile_list<C::R>(p, list, list + C::kListInts, n_rounds);
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(smem_addr(&bars->q_full), kTileM);
@@ -271,10 +349,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t item = 0;
       bool ok = true;
-      for (int r = 0; r * int(gridDim.x) < p.num_tiles && ok; ++r) {
-        const int tile = snake_tile(r);
-        if (tile >= p.num_tiles) continue;
-        const TileInfo t = tile_info<C::R>(p, tile);
+      for (int r = 0; r < n_rounds && ok; ++r) {
+        int tile_row;
+        if (!round_tile<C::R>(p, list, r, tile_row)) continue;
+        const TileInfo t = tile_info<C::R>(p, tile_row);
         if (union_count(t, p.words) == 0) continue;
         CrmIter it;
         it.init(t.row0, t.row1, p.words);
@@ -363,10 +441,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         return wait_fast(smem_addr(&bars->kv_full[it % C::kStages]), (it / C::kStages) & 1,
                             abort);
       };
-      for (int r = 0; r * int(gridDim.x) < p.num_tiles && ok; ++r) {
-        const int tile = snake_tile(r);
-        if (tile >= p.num_tiles) continue;
-        const TileInfo t = tile_info<C::R>(p, tile);
+      for (int r = 0; r < n_rounds && ok; ++r) {
+        int tile_row;
+        if (!round_tile<C::R>(p, list, r, tile_row)) continue;
+        const TileInfo t = tile_info<C::R>(p, tile_row);
         const int kept = union_count(t, p.words);
         if (kept == 0) continue;
         const int cnt = C::kPairs ? (kept + 1) / 2 : kept;  // S tiles of this query tile
@@ -416,10 +494,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t g = 0;
     bool ok = true;
     const bool has_tail = p.n_valid < p.n_pad;
-    for (int r = 0; r * int(gridDim.x) < p.num_tiles && ok; ++r) {
-      const int tile = snake_tile(r);
-      if (tile >= p.num_tiles) continue;
-      const TileInfo t = tile_info<C::R>(p, tile);
+    for (int r = 0; r < n_rounds && ok; ++r) {
+      int tile_row;
+      if (!round_tile<C::R>(p, list, r, tile_row)) continue;
+      const TileInfo t = tile_info<C::R>(p, tile_row);
       const int my_qb = t.qb0 + row / BQ;
       const bool row_in_head = my_qb < p.nb_q;
       const uint32_t* my_bits = p.bits + (int64_t(t.bh) * p.nb_q + my_qb) * p.words;
@@ -716,6 +794,7 @@ bsa_status launch_forward(const void* q, const void* k, const void* v, const bsa
   const int sms = bsa::num_sms();
   if (sms <= 0) return BSA_ERR_LAUNCH;
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  p.use_list = (C::R > 1 && (p.num_tiles + grid - 1) / grid <= C::kListInts) ? 1 : 0;
   bsa_forward_kernel<D, BQ, BK><<<grid, kThreads, C::kSmemBytes, stream>>>(tk, tv, p);
   return bsa::launch_status();
 }

@@ -85,12 +85,16 @@ const char* bsa_status_string(bsa_status status);
  *               ordered by counts descending; equal counts keep ascending r.
  *               Then the order is checked for how many heads it mixes: over
  *               its full windows of 148 consecutive entries (one wave of a
- *               B200), if the distinct heads h' = r / nb_q (one per (b, h))
- *               total more than 8 per window, the schedule is instead ordered
+ *               B200), the distinct heads h' = r / nb_q (one per (b, h)) are
+ *               counted; if that many heads' K and V (nb_k key blocks each,
+ *               costed as 128 tokens at d = 128 in bf16: 64 KiB) exceed the
+ *               device's L2 size on average, the schedule is instead ordered
  *               by head h' ascending, then counts descending, then r
  *               ascending.  (Query tiles taken together then share one head's
  *               K and V in L2; the check is skipped, keeping the count
- *               order, when B*H > 8192 or nb_q > 8192.)
+ *               order, when B*H > 8192 or nb_q > 8192.)  Any order gives the
+ *               same attention output; the forward only takes it as its work
+ *               order.
  *   workspace   device scratch of at least bsa_pack_mask_workspace(...) bytes,
  *               16-byte aligned; its contents on entry do not matter.
  *
