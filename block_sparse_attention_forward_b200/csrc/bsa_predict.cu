@@ -17,14 +17,17 @@
 //   1. pool:        one CTA per (b, h, block); fp32 means of the block's
 //                   valid q and k rows into the workspace (HBM bound: q and k
 //                   are read once).
-//   2. score_topp:  one CTA per (b, h, kRowsPerCta query blocks).  Scores by
-//                   fp32 FMA in 4 x 4 register tiles against key means staged
-//                   in shared memory; then one warp per row: max, exp, sum, and the cut
-//                   found by bisection on the bit patterns of the
-//                   (non-negative) exponentials -- the largest T with
+//   2. score_tile:  one CTA per (b, h, 32 query blocks).  Scores by fp32 FMA
+//                   in 8 x 4 register tiles against key means staged in
+//                   shared memory by cp.async, two slices deep, into a
+//                   [B*H, nb, nb] fp32 buffer in the workspace (L2-resident at
+//                   the workloads' sizes).
+//   3. topp_rows:   one warp per row: max, exp, sum, and the cut found by
+//                   bisection on the bit patterns of the (non-negative)
+//                   exponentials -- the largest T with
 //                   sum(e_j >= T) >= top_p * sum(e) -- then ties at T taken
 //                   in index order; the kept blocks are balloted into CRM words.
-//   3-6. the tiled count sort and the kept-block lists shared with packing.
+//   4-8. the tiled count sort and the kept-block lists shared with packing.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -34,7 +37,6 @@
 namespace {
 
 constexpr int kPoolThreads = 256;
-constexpr int kRowsPerCta = 16;  // query blocks per score CTA
 constexpr int kKeyChunk = 256;   // key blocks per pass
 constexpr int kDSlice = 32;      // dimensions of the key means staged at a time
 constexpr int kKsStride = kDSlice + 4;  // padded row (16-byte aligned, conflict-free)
@@ -116,7 +118,7 @@ __device__ __forceinline__ int warp_sum_int(int x) {
 // reaches it (top_p >= 1, or rounding) every block is kept.  Block j = l + 32 k
 // is bit l of CRM word k.
 template <int kPerLane>
-__device__ __forceinline__ void top_p_row(float* __restrict__ s_row, int nb, float p_h,
+__device__ __forceinline__ void top_p_row(const float* __restrict__ s_row, int nb, float p_h,
                                           uint32_t* __restrict__ out,
                                           int32_t* __restrict__ count) {
   const int lane = threadIdx.x & 31;
@@ -180,104 +182,152 @@ __device__ __forceinline__ void top_p_row(float* __restrict__ s_row, int nb, flo
   if (lane == 0) *count = total;
 }
 
-// Dynamic shared memory: qs [kRowsPerCta][d] | ks [kKeyChunk][kKsStride] |
-// sc [kRowsPerCta][nb] (scores, then exponentials).  blockIdx.x = group of
-// kRowsPerCta query blocks, blockIdx.y = b*H + h.  Scores: thread t owns a
-// 4 x 4 tile -- rows 4 (t / 64) + a, keys (t % 64) + 64 b of each pass -- and
-// reads 16-byte vectors of the query means (broadcast within a warp) and of
-// the staged key means (a padded row stride keeps a quarter warp's vectors in
-// distinct banks): 8 vector loads per 64 FMAs.
-template <int kPerLane>
+// Scores alone, written to a global [B*H, nb, nb] buffer (L2-resident at the
+// workloads' sizes): one CTA per (b, h, 32 query blocks), each thread an
+// 8-row x 4-key register tile (rows 8 (t / 64) + a, keys (t % 64) + 64 b of
+// each pass of kKeyChunk keys), so that one 16-byte vector of key means (a
+// quarter warp's in distinct banks) feeds 8 FMA chains and one broadcast
+// vector of query means feeds 4: 12 vector loads per 128 FMAs.  The key means
+// are staged 32 dimensions at a time, the next slice's cp.async copies in
+// flight while this slice's FMAs run.  88 KB of shared memory: two CTAs per SM.
+constexpr int kRowsTile = 32;
+constexpr int kSliceFloats = kKeyChunk * kKsStride;  // one staged slice of key means
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __global__ void __launch_bounds__(kScoreThreads)
-    score_topp_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar, int H,
-                      int nb, int d, const float* __restrict__ tau,
-                      const float* __restrict__ top_p, uint32_t* __restrict__ bits,
-                      int32_t* __restrict__ counts) {
+    score_tile_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar, int H,
+                      int nb, int d, const float* __restrict__ tau, float* __restrict__ scores) {
   extern __shared__ float4 score_smem4[];
-  float* qs = reinterpret_cast<float*>(score_smem4);
-  float* ks = qs + kRowsPerCta * d;
-  float* sc = ks + kKeyChunk * kKsStride;
+  float* qs = reinterpret_cast<float*>(score_smem4);  // [kRowsTile][d]
+  float* ks = qs + kRowsTile * d;                     // [2][kKeyChunk][kKsStride]
   const int64_t bh = blockIdx.y;
   const int h = int(bh % H);
-  const int i0 = blockIdx.x * kRowsPerCta;
-  const int rows = min(kRowsPerCta, nb - i0);
+  const int i0 = blockIdx.x * kRowsTile;
+  const int rows = min(kRowsTile, nb - i0);
   const float inv_denom = 1.0f / (sqrtf(float(d)) * __ldg(tau + h));
+  const int slices_per_chunk = d / kDSlice;
+  const int n_slices = ((nb + kKeyChunk - 1) / kKeyChunk) * slices_per_chunk;
 
-  for (int e = threadIdx.x; e < kRowsPerCta * d; e += kScoreThreads) {
+  // slice sl = (key chunk sl / slices_per_chunk, dims 32 (sl % slices_per_chunk))
+  // into buffer sl & 1: 256 keys x 8 vectors, 8 per thread; keys past nb read
+  // zeros (source size 0)
+  auto stage = [&](int sl) {
+    const int j0 = (sl / slices_per_chunk) * kKeyChunk;
+    const int c0 = (sl % slices_per_chunk) * kDSlice;
+    float* buf = ks + (sl & 1) * kSliceFloats;
+    for (int e = threadIdx.x; e < kKeyChunk * (kDSlice / 4); e += kScoreThreads) {
+      const int key = e / (kDSlice / 4), part = e - key * (kDSlice / 4);
+      const bool in = j0 + key < nb;
+      const float* src = kbar + ((bh * nb + (in ? j0 + key : 0)) * d + c0 + part * 4);
+      cp_async16(static_cast<uint32_t>(__cvta_generic_to_shared(buf + key * kKsStride + part * 4)),
+                 src, in ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+
+  stage(0);
+  for (int e = threadIdx.x; e < kRowsTile * d; e += kScoreThreads) {
     const int r = e / d, c = e - r * d;
     qs[e] = r < rows ? qbar[(bh * nb + i0 + r) * d + c] : 0.0f;
   }
   const int rg = threadIdx.x / 64, kg = threadIdx.x % 64;
-  const float4* kbar4 = reinterpret_cast<const float4*>(kbar);
-  for (int j0 = 0; j0 < nb; j0 += kKeyChunk) {
-    const int keys = min(kKeyChunk, nb - j0);
-    float acc[4][4] = {};
-    for (int c0 = 0; c0 < d; c0 += kDSlice) {
-      __syncthreads();  // the previous slice's reads of ks are done; qs is staged
-      for (int e = threadIdx.x; e < kKeyChunk * (kDSlice / 4); e += kScoreThreads) {
-        const int key = e / (kDSlice / 4), part = e - key * (kDSlice / 4);
-        const float4 v = key < keys ? __ldg(kbar4 + ((bh * nb + j0 + key) * d + c0) / 4 + part)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4*>(ks + key * kKsStride + part * 4) = v;
-      }
-      __syncthreads();
+  float acc[8][4];
 #pragma unroll
-      for (int c4 = 0; c4 < kDSlice / 4; ++c4) {
-        float4 qv[4], kv[4];
+  for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
-          qv[a] = *reinterpret_cast<const float4*>(qs + (rg * 4 + a) * d + c0 + c4 * 4);
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+  for (int sl = 0; sl < n_slices; ++sl) {
+    if (sl + 1 < n_slices) {
+      stage(sl + 1);
+      cp_async_wait<1>();  // this slice has landed (the next may be in flight)
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const int c0 = (sl % slices_per_chunk) * kDSlice;
+    const float* buf = ks + (sl & 1) * kSliceFloats;
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
-          kv[b] = *reinterpret_cast<const float4*>(ks + (kg + 64 * b) * kKsStride + c4 * 4);
+    for (int c4 = 0; c4 < kDSlice / 4; ++c4) {
+      float4 qv[8], kv[4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+      for (int a = 0; a < 8; ++a)
+        qv[a] = *reinterpret_cast<const float4*>(qs + (rg * 8 + a) * d + c0 + c4 * 4);
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            acc[a][b] = fmaf(qv[a].x, kv[b].x, acc[a][b]);
-            acc[a][b] = fmaf(qv[a].y, kv[b].y, acc[a][b]);
-            acc[a][b] = fmaf(qv[a].z, kv[b].z, acc[a][b]);
-            acc[a][b] = fmaf(qv[a].w, kv[b].w, acc[a][b]);
-          }
+      for (int b = 0; b < 4; ++b)
+        kv[b] = *reinterpret_cast<const float4*>(buf + (kg + 64 * b) * kKsStride + c4 * 4);
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          acc[a][b] = fmaf(qv[a].x, kv[b].x, acc[a][b]);
+          acc[a][b] = fmaf(qv[a].y, kv[b].y, acc[a][b]);
+          acc[a][b] = fmaf(qv[a].z, kv[b].z, acc[a][b]);
+          acc[a][b] = fmaf(qv[a].w, kv[b].w, acc[a][b]);
+        }
+    }
+    if (sl % slices_per_chunk == slices_per_chunk - 1) {  // a key chunk is complete
+      const int j0 = (sl / slices_per_chunk) * kKeyChunk;
+#pragma unroll
+      for (int a = 0; a < 8; ++a) {
+        const int r = rg * 8 + a;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int key = j0 + kg + 64 * b;
+          if (r < rows && key < nb) scores[(bh * nb + i0 + r) * nb + key] = acc[a][b] * inv_denom;
+          acc[a][b] = 0.0f;
+        }
       }
     }
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int key = kg + 64 * b;
-        if (key < keys) sc[(rg * 4 + a) * nb + j0 + key] = acc[a][b] * inv_denom;
-      }
+    __syncthreads();  // every thread is done with this buffer before it is refilled
   }
-  __syncthreads();
-
-  const int warp = threadIdx.x >> 5;
-  const float p_h = __ldg(top_p + h);
-  for (int rr = warp; rr < rows; rr += kScoreThreads / 32)
-    top_p_row<kPerLane>(sc + rr * nb, nb, p_h, bits + (bh * nb + i0 + rr) * ((nb + 31) / 32),
-                        counts + bh * nb + i0 + rr);
 }
 
-size_t score_smem_bytes(int nb, int d) {
-  return sizeof(float) * (size_t(kRowsPerCta) * d + size_t(kKeyChunk) * kKsStride +
-                          size_t(kRowsPerCta) * nb);
+// The cut, one warp per row of the score buffer (kScoreThreads / 32 rows per CTA).
+template <int kPerLane>
+__global__ void __launch_bounds__(kScoreThreads)
+    topp_rows_kernel(const float* __restrict__ scores, int H, int nb, int rows,
+                     const float* __restrict__ top_p, uint32_t* __restrict__ bits,
+                     int32_t* __restrict__ counts) {
+  const int r = blockIdx.x * (kScoreThreads / 32) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const int h = (r / nb) % H;
+  top_p_row<kPerLane>(scores + int64_t(r) * nb, nb, __ldg(top_p + h),
+                      bits + int64_t(r) * ((nb + 31) / 32), counts + r);
+}
+
+size_t score_tile_smem_bytes(int d) {
+  return sizeof(float) * (size_t(kRowsTile) * d + 2 * size_t(kSliceFloats));
+}
+
+size_t scores_bytes(int64_t BH, int nb) {
+  const size_t b = size_t(BH) * nb * nb * sizeof(float);
+  return (b + 255) & ~size_t(255);
+}
+
+template <int kPerLane>
+bsa_status launch_topp_rows(int rows, cudaStream_t s, const float* scores, int H, int nb,
+                            const float* top_p, uint32_t* bits, int32_t* counts) {
+  const int per_cta = kScoreThreads / 32;
+  topp_rows_kernel<kPerLane><<<(rows + per_cta - 1) / per_cta, kScoreThreads, 0, s>>>(
+      scores, H, nb, rows, top_p, bits, counts);
+  return bsa::launch_status() == BSA_OK ? BSA_OK : BSA_ERR_LAUNCH;
 }
 
 size_t means_bytes(int64_t BH, int nb, int d) {
   const size_t b = size_t(BH) * nb * d * sizeof(float);
   return (b + 255) & ~size_t(255);
-}
-
-template <int kPerLane>
-bsa_status launch_score(dim3 grid, size_t smem, cudaStream_t s, const float* qbar,
-                        const float* kbar, int H, int nb, int d, const float* tau,
-                        const float* top_p, uint32_t* bits, int32_t* counts) {
-  if (cudaFuncSetAttribute(score_topp_kernel<kPerLane>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-    return BSA_ERR_LAUNCH;
-  score_topp_kernel<kPerLane><<<grid, kScoreThreads, smem, s>>>(qbar, kbar, H, nb, d, tau, top_p,
-                                                                bits, counts);
-  return bsa::launch_status() == BSA_OK ? BSA_OK : BSA_ERR_LAUNCH;
 }
 
 }  // namespace
@@ -286,7 +336,7 @@ extern "C" size_t bsa_predict_top_p_workspace(int B, int H, int n_pad, int d, in
   if (B <= 0 || H <= 0 || n_pad <= 0 || d <= 0 || block <= 0 || n_pad % block != 0) return 0;
   const int nb = n_pad / block;
   const int64_t BH = int64_t(B) * H;
-  return 2 * means_bytes(BH, nb, d) + bsa::pack_scratch_bytes(BH * nb, nb);
+  return 2 * means_bytes(BH, nb, d) + scores_bytes(BH, nb) + bsa::pack_scratch_bytes(BH * nb, nb);
 }
 
 extern "C" bsa_status bsa_predict_top_p(const void* q, const void* k, int B, int H, int n_valid,
@@ -320,26 +370,33 @@ extern "C" bsa_status bsa_predict_top_p(const void* q, const void* k, int B, int
   char* ws = static_cast<char*>(workspace);
   float* qbar = reinterpret_cast<float*>(ws);
   float* kbar = reinterpret_cast<float*>(ws + means_bytes(BH, nb, d));
-  void* scratch = ws + 2 * means_bytes(BH, nb, d);
+  float* scores = reinterpret_cast<float*>(ws + 2 * means_bytes(BH, nb, d));
+  void* scratch = ws + 2 * means_bytes(BH, nb, d) + scores_bytes(BH, nb);
 
   pool_kernel<<<dim3(unsigned(nb), unsigned(BH)), kPoolThreads, 0, s>>>(
       static_cast<const uint4*>(q), static_cast<const uint4*>(k), n_valid, n_pad, d, block, qbar,
       kbar);
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
-  const size_t smem = score_smem_bytes(nb, d);
-  const dim3 grid(unsigned((nb + kRowsPerCta - 1) / kRowsPerCta), unsigned(BH));
+  const size_t smem = score_tile_smem_bytes(d);
+  if (cudaFuncSetAttribute(score_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(smem)) != cudaSuccess)
+    return BSA_ERR_LAUNCH;
+  score_tile_kernel<<<dim3(unsigned((nb + kRowsTile - 1) / kRowsTile), unsigned(BH)),
+                      kScoreThreads, smem, s>>>(qbar, kbar, H, nb, d, tau, scores);
+  if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
+  const int rows = int(BH * nb);
   const int per_lane = (nb + 31) / 32;
   bsa_status st;
   if (per_lane <= 8)
-    st = launch_score<8>(grid, smem, s, qbar, kbar, H, nb, d, tau, top_p, bits, counts);
+    st = launch_topp_rows<8>(rows, s, scores, H, nb, top_p, bits, counts);
   else if (per_lane <= 16)
-    st = launch_score<16>(grid, smem, s, qbar, kbar, H, nb, d, tau, top_p, bits, counts);
+    st = launch_topp_rows<16>(rows, s, scores, H, nb, top_p, bits, counts);
   else if (per_lane <= 20)
-    st = launch_score<20>(grid, smem, s, qbar, kbar, H, nb, d, tau, top_p, bits, counts);
+    st = launch_topp_rows<20>(rows, s, scores, H, nb, top_p, bits, counts);
   else if (per_lane <= 32)
-    st = launch_score<32>(grid, smem, s, qbar, kbar, H, nb, d, tau, top_p, bits, counts);
+    st = launch_topp_rows<32>(rows, s, scores, H, nb, top_p, bits, counts);
   else
-    st = launch_score<64>(grid, smem, s, qbar, kbar, H, nb, d, tau, top_p, bits, counts);
+    st = launch_topp_rows<64>(rows, s, scores, H, nb, top_p, bits, counts);
   if (st != BSA_OK) return st;
   return bsa::pack_finish(bits, counts, int(BH * nb), nb, nb, row_offsets, col_idx, schedule, scratch,
                           s);

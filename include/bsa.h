@@ -243,7 +243,8 @@ bsa_status bsa_tile_unpermute(const void* in, void* out, int B, int H, int T, in
  *   bits, counts, row_offsets, col_idx, schedule: as for bsa_pack_mask with
  *             nb_q = nb_k = n_pad / block.
  *   workspace device scratch of bsa_predict_top_p_workspace(...) bytes,
- *             16-byte aligned (pooled means and the sort's tables).
+ *             16-byte aligned (pooled means, the fp32 block scores
+ *             [B*H, nb, nb] and the sort's tables).
  *
  * Supported: d in {64, 128}; n_pad % block == 0; n_pad - block < n_valid <=
  * n_pad; n_pad / block <= 2048; B*H <= 65535.  Errors: BSA_ERR_INVALID_ARG,
