@@ -85,6 +85,10 @@ SMALL = [
                                                8, 16, 128, 15, "bernoulli_sparse")),
     ("band_stripe_small", I.custom_workload("band_stripe_small", 1, 3, 128, 5, 30, 52, 1, 8, 16,
                                             128, 16, "band_stripe")),
+    # 64-token blocks, 8 heads x 32 tiles of two blocks: more tiles than SMs, so every
+    # CTA takes tiles from its schedule-ordered list over two rounds
+    ("d64_b64_two_rounds", I.custom_workload("d64_b64_two_rounds", 1, 8, 64, 4, 32, 32, 1, 8, 8,
+                                             64, 18, "bernoulli_half")),
 ]
 
 

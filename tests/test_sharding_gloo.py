@@ -85,3 +85,24 @@ def test_rank_slices_cover_every_head_once(name):
             lo, hi = head_range(w.B * w.H, world, rank)
             seen[lo:hi] += 1
         assert np.all(seen == 1), (name, world)
+
+
+def test_bench_shard_workload_slices_reassemble():
+    # bench.py --gpus N: each rank's slice of q, k, v and mask, concatenated in
+    # rank order, is the whole problem
+    import importlib.util
+    from block_sparse_attention_forward_b200 import inputs as I
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(root, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    w = I.custom_workload("shard", 2, 3, 64, 2, 8, 8, 1, 8, 8, 64, 5, "bernoulli_half")
+    q, k, v = I.gen_qkv(w)
+    mask = I.gen_mask(w)
+    for world in (1, 2, 4):
+        parts = [bench.shard_workload(w, q, k, v, mask, world, r) for r in range(world)]
+        assert sum(p[0].H for p in parts) == w.B * w.H
+        got_q = torch.cat([p[1] for p in parts], dim=1).reshape(q.shape)
+        got_m = np.concatenate([p[4] for p in parts], axis=1).reshape(mask.shape)
+        assert torch.equal(got_q, q)
+        assert np.array_equal(got_m, mask)
