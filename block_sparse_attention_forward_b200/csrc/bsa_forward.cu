@@ -865,6 +865,9 @@ extern "C" bsa_status bsa_get_device_error(bsa_status* device_status) {
     return BSA_ERR_LAUNCH;
   if (cudaMemcpyToSymbol(g_bsa_device_error, &zero, sizeof(int)) != cudaSuccess)
     return BSA_ERR_LAUNCH;
+  const int pred = bsa::take_predict_device_error();
+  if (pred < 0) return BSA_ERR_LAUNCH;
+  if (host == 0) host = pred;
   *device_status = host == 0 ? BSA_OK : bsa_status(host);
   return BSA_OK;
 }

@@ -36,4 +36,9 @@ bsa_status pack_finish(const uint32_t* bits, const int32_t* counts, int rows, in
 // Largest nb_k the packing stages accept (BSA_ERR_UNSUPPORTED beyond).
 constexpr int kPackMaxNbK = 49151;
 
+// The predictor's device-side error word (BSA_ERR_TIMEOUT after a wait of its
+// score kernel ran out, else 0), read and cleared; -1 if the copy failed.
+// Defined in bsa_predict.cu.
+int take_predict_device_error();
+
 }  // namespace bsa

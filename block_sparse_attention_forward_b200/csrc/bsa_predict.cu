@@ -17,31 +17,44 @@
 //   1. pool:        one CTA per (b, h, block); fp32 means of the block's
 //                   valid q and k rows into the workspace (HBM bound: q and k
 //                   are read once).
-//   2. score_tile:  one CTA per (b, h, 32 query blocks).  Scores by fp32 FMA
-//                   in 8 x 4 register tiles against key means staged in
-//                   shared memory by cp.async, two slices deep, into a
+//   2. score_mma:   one CTA per (b, h, 128 query blocks, 64 key blocks): the
+//                   contraction qbar kbar^T on the tensor cores
+//                   (tcgen05.mma kind::tf32, accumulator in TMEM).  Each mean
+//                   is split into a tf32 part (its 13 low mantissa bits
+//                   cleared) and the exact remainder, and the scores are the
+//                   three products hi.hi + hi.lo + lo.hi, which carry
+//                   fp32-level accuracy (the dropped lo.lo term and the tf32
+//                   rounding of the remainders are below 2^-19 of each
+//                   product).  TMA loads 32 dimensions at a time into a
+//                   2-stage ring, where the CTA's threads split them in place;
+//                   the scaled scores go through shared memory to a
 //                   [B*H, nb, nb] fp32 buffer in the workspace (L2-resident at
-//                   the workloads' sizes).
+//                   the workloads' sizes) in coalesced rows.
 //   3. topp_rows:   one warp per row: max, exp, sum, and the cut found by
 //                   bisection on the bit patterns of the (non-negative)
 //                   exponentials -- the largest T with
 //                   sum(e_j >= T) >= top_p * sum(e) -- then ties at T taken
 //                   in index order; the kept blocks are balloted into CRM words.
 //   4-8. the tiled count sort and the kept-block lists shared with packing.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "bsa.h"
 #include "bsa_internal.h"
+#include "sm100_ptx.cuh"
+
+// BSA_ERR_TIMEOUT when a wait of the score kernel ran out (read and cleared by
+// bsa_get_device_error through bsa::take_predict_device_error)
+__device__ int g_predict_device_error = 0;
 
 namespace {
 
+using namespace sm100;
+
 constexpr int kPoolThreads = 256;
-constexpr int kKeyChunk = 256;   // key blocks per pass
-constexpr int kDSlice = 32;      // dimensions of the key means staged at a time
-constexpr int kKsStride = kDSlice + 4;  // padded row (16-byte aligned, conflict-free)
 constexpr int kScoreThreads = 256;
-constexpr int kMaxBlocks = 2048;  // nb limit: the score rows live in shared memory
+constexpr int kMaxBlocks = 2048;  // nb limit of the cut (score rows per warp in registers)
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -182,115 +195,220 @@ __device__ __forceinline__ void top_p_row(const float* __restrict__ s_row, int n
   if (lane == 0) *count = total;
 }
 
-// Scores alone, written to a global [B*H, nb, nb] buffer (L2-resident at the
-// workloads' sizes): one CTA per (b, h, 32 query blocks), each thread an
-// 8-row x 4-key register tile (rows 8 (t / 64) + a, keys (t % 64) + 64 b of
-// each pass of kKeyChunk keys), so that one 16-byte vector of key means (a
-// quarter warp's in distinct banks) feeds 8 FMA chains and one broadcast
-// vector of query means feeds 4: 12 vector loads per 128 FMAs.  The key means
-// are staged 32 dimensions at a time, the next slice's cp.async copies in
-// flight while this slice's FMAs run.  88 KB of shared memory: two CTAs per SM.
-constexpr int kRowsTile = 32;
-constexpr int kSliceFloats = kKeyChunk * kKsStride;  // one staged slice of key means
+// Scores on the tensor cores: one CTA of 128 threads per (b, h, 128 query
+// blocks i0.., 64 key blocks j0..), two CTAs per SM (97 KB of shared memory
+// each), so that one CTA's loads and stores overlap the other's products.
+// Thread 0 issues the TMA loads of the means, 32 dimensions (one 128-byte
+// swizzle atom per row) per stage: query means 16 KB, key means 8 KB; all
+// 128 threads then split each value in place
+// into its tf32 part and write the remainder at the same offset of a parallel
+// region (the split is elementwise, so the swizzle carries over); thread 32
+// issues per stage 4 steps of K = 8, each three tcgen05.mma kind::tf32
+// products into one 128 x 64 fp32 accumulator in TMEM (hi.hi, hi.lo, lo.hi);
+// all four warps then move the accumulator (one query block per TMEM lane)
+// through shared memory to the score rows.  Rows or keys past nb (the next head's, or the
+// zero fill past the last head) are computed and not stored.
+constexpr int kMmaThreads = 128;
+constexpr int kTileK = 64;                                // key blocks per CTA
+constexpr uint32_t kQPart = 128u * 128u;                  // 128 query rows x 32 fp32
+constexpr uint32_t kKPart = uint32_t(kTileK) * 128u;     // 64 key rows x 32 fp32
+constexpr uint32_t kLoaded = kQPart + kKPart;             // q, k as loaded
+constexpr uint32_t kStageBytes = 2u * kLoaded;            // q hi, k hi, q lo, k lo
+constexpr int kMmaStages = 2;
+constexpr int kOutStride = kTileK + 1;                    // floats per staged output row
+constexpr uint64_t kScoreTimeoutNs = 2000000000ull;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
+struct ScoreBars {
+  uint64_t full[kMmaStages], split[kMmaStages], empty[kMmaStages], done;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kScoreMmaSmem = size_t(kMmaStages) * kStageBytes + 256 + 1024;
+static_assert(size_t(128) * kOutStride * 4 <= size_t(kMmaStages) * kStageBytes, "output staging");
+static_assert(kQPart % 1024 == 0 && kLoaded % 1024 == 0, "1024-byte aligned swizzled tiles");
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::tf32 (fp32 containers, fp32 accumulate)
+__device__ __forceinline__ void mma_ss_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
+
+// Instruction descriptor, kind::tf32: fp32 accumulator (bits 4-5 = 1), tf32 A
+// and B (bits 7-9 = 2, bits 10-12 = 2), both K-major, N >> 3 at bits 17-22,
+// M >> 4 at bits 24-28.
+constexpr uint32_t idesc_tf32_f32(int M, int N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
-__global__ void __launch_bounds__(kScoreThreads)
-    score_tile_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar, int H,
-                      int nb, int d, const float* __restrict__ tau, float* __restrict__ scores) {
-  extern __shared__ float4 score_smem4[];
-  float* qs = reinterpret_cast<float*>(score_smem4);  // [kRowsTile][d]
-  float* ks = qs + kRowsTile * d;                     // [2][kKeyChunk][kKsStride]
-  const int64_t bh = blockIdx.y;
-  const int h = int(bh % H);
-  const int i0 = blockIdx.x * kRowsTile;
-  const int rows = min(kRowsTile, nb - i0);
-  const float inv_denom = 1.0f / (sqrtf(float(d)) * __ldg(tau + h));
-  const int slices_per_chunk = d / kDSlice;
-  const int n_slices = ((nb + kKeyChunk - 1) / kKeyChunk) * slices_per_chunk;
-
-  // slice sl = (key chunk sl / slices_per_chunk, dims 32 (sl % slices_per_chunk))
-  // into buffer sl & 1: 256 keys x 8 vectors, 8 per thread; keys past nb read
-  // zeros (source size 0)
-  auto stage = [&](int sl) {
-    const int j0 = (sl / slices_per_chunk) * kKeyChunk;
-    const int c0 = (sl % slices_per_chunk) * kDSlice;
-    float* buf = ks + (sl & 1) * kSliceFloats;
-    for (int e = threadIdx.x; e < kKeyChunk * (kDSlice / 4); e += kScoreThreads) {
-      const int key = e / (kDSlice / 4), part = e - key * (kDSlice / 4);
-      const bool in = j0 + key < nb;
-      const float* src = kbar + ((bh * nb + (in ? j0 + key : 0)) * d + c0 + part * 4);
-      cp_async16(static_cast<uint32_t>(__cvta_generic_to_shared(buf + key * kKsStride + part * 4)),
-                 src, in ? 16u : 0u);
-    }
-    cp_async_commit();
-  };
-
-  stage(0);
-  for (int e = threadIdx.x; e < kRowsTile * d; e += kScoreThreads) {
-    const int r = e / d, c = e - r * d;
-    qs[e] = r < rows ? qbar[(bh * nb + i0 + r) * d + c] : 0.0f;
-  }
-  const int rg = threadIdx.x / 64, kg = threadIdx.x % 64;
-  float acc[8][4];
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-  for (int sl = 0; sl < n_slices; ++sl) {
-    if (sl + 1 < n_slices) {
-      stage(sl + 1);
-      cp_async_wait<1>();  // this slice has landed (the next may be in flight)
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const int c0 = (sl % slices_per_chunk) * kDSlice;
-    const float* buf = ks + (sl & 1) * kSliceFloats;
-#pragma unroll
-    for (int c4 = 0; c4 < kDSlice / 4; ++c4) {
-      float4 qv[8], kv[4];
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-        qv[a] = *reinterpret_cast<const float4*>(qs + (rg * 8 + a) * d + c0 + c4 * 4);
-#pragma unroll
-      for (int b = 0; b < 4; ++b)
-        kv[b] = *reinterpret_cast<const float4*>(buf + (kg + 64 * b) * kKsStride + c4 * 4);
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          acc[a][b] = fmaf(qv[a].x, kv[b].x, acc[a][b]);
-          acc[a][b] = fmaf(qv[a].y, kv[b].y, acc[a][b]);
-          acc[a][b] = fmaf(qv[a].z, kv[b].z, acc[a][b]);
-          acc[a][b] = fmaf(qv[a].w, kv[b].w, acc[a][b]);
-        }
-    }
-    if (sl % slices_per_chunk == slices_per_chunk - 1) {  // a key chunk is complete
-      const int j0 = (sl / slices_per_chunk) * kKeyChunk;
-#pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        const int r = rg * 8 + a;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int key = j0 + kg + 64 * b;
-          if (r < rows && key < nb) scores[(bh * nb + i0 + r) * nb + key] = acc[a][b] * inv_denom;
-          acc[a][b] = 0.0f;
-        }
+// Bounded wait: true once the phase of `parity` completed; false after about
+// two seconds (records BSA_ERR_TIMEOUT) or, with abort != nullptr, when
+// another thread of the CTA gave up.
+__device__ __noinline__ bool score_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (abort && *abort) return false;
+      if (global_timer_ns() - t0 > kScoreTimeoutNs) {
+        if (abort) *abort = 1;
+        atomicExch(&g_predict_device_error, int(BSA_ERR_TIMEOUT));
+        return false;
       }
     }
-    __syncthreads();  // every thread is done with this buffer before it is refilled
+  }
+}
+
+__global__ void __launch_bounds__(kMmaThreads, 1)
+    score_mma_kernel(const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_k, int H, int nb, int d,
+                     const float* __restrict__ tau, float* __restrict__ scores) {
+  extern __shared__ __align__(1024) uint8_t score_smem_raw[];
+  // 128-byte swizzle atoms need 1024-byte aligned tiles
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(score_smem_raw) + 1023) & ~uintptr_t(1023));
+  ScoreBars* bars = reinterpret_cast<ScoreBars*>(smem + size_t(kMmaStages) * kStageBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j0 = blockIdx.x * kTileK, i0 = blockIdx.y * 128;
+  const int bh = blockIdx.z;
+  const int n_st = d / 32;  // stages of 32 dimensions
+  volatile int* abort = &bars->abort;
+  const uint32_t s0 = smem_addr(smem);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMmaStages; ++i) {
+      mbar_init(smem_addr(&bars->full[i]), 1);
+      mbar_init(smem_addr(&bars->split[i]), kMmaThreads);
+      mbar_init(smem_addr(&bars->empty[i]), 1);
+    }
+    mbar_init(smem_addr(&bars->done), 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&bars->tmem_base), kTileK);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  // Per stage st (slot st % kMmaStages): thread 0 loads it (the first
+  // kMmaStages up front, stage st + kMmaStages once the products of stage st
+  // have released the slot); every thread splits it once it has landed and
+  // arrives on `split`; thread 32 issues its products once all 128 have.
+  constexpr uint32_t idesc = idesc_tf32_f32(128, kTileK);
+  auto load_stage = [&](int st) {
+    const int slot = st % kMmaStages;
+    const uint32_t fbar = smem_addr(&bars->full[slot]);
+    mbar_arrive_expect_tx(fbar, kLoaded);
+    const uint32_t base = s0 + slot * kStageBytes;
+    tma_load_2d(base, &tm_q, fbar, st * 32, bh * nb + i0);
+    tma_load_2d(base + kQPart, &tm_k, fbar, st * 32, bh * nb + j0);
+  };
+  if (threadIdx.x == 0)
+    for (int st = 0; st < n_st && st < kMmaStages; ++st) load_stage(st);
+  bool ok = true;
+  for (int st = 0; st < n_st; ++st) {
+    const int slot = st % kMmaStages;
+    const uint32_t par = (st / kMmaStages) & 1;
+    // ---------------------------------------------------------- split
+    // the stage's 24 KB of means -> tf32 parts in place, exact remainders
+    // 24 KB further
+    ok = ok && score_wait(smem_addr(&bars->full[slot]), par, abort);
+    if (ok) {
+      uint4* v = reinterpret_cast<uint4*>(smem + size_t(slot) * kStageBytes);
+      uint4* lo = v + kLoaded / 16;
+      for (int e = threadIdx.x; e < int(kLoaded / 16); e += kMmaThreads) {
+        const uint4 x = v[e];
+        uint4 h, r;
+        h.x = x.x & 0xFFFFE000u; r.x = __float_as_uint(__uint_as_float(x.x) - __uint_as_float(h.x));
+        h.y = x.y & 0xFFFFE000u; r.y = __float_as_uint(__uint_as_float(x.y) - __uint_as_float(h.y));
+        h.z = x.z & 0xFFFFE000u; r.z = __float_as_uint(__uint_as_float(x.z) - __uint_as_float(h.z));
+        h.w = x.w & 0xFFFFE000u; r.w = __float_as_uint(__uint_as_float(x.w) - __uint_as_float(h.w));
+        v[e] = h;
+        lo[e] = r;
+      }
+      // generic-proxy writes of shared memory become visible to the tensor core
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    // arrive even after a failure, so that the MMA issuer's wait ends
+    mbar_arrive(smem_addr(&bars->split[slot]));
+    if (threadIdx.x == 32) {
+      // -------------------------------------------------------- MMA issuer
+      if (score_wait(smem_addr(&bars->split[slot]), par, nullptr)) {
+        tc_fence_after();
+        const uint32_t base = s0 + slot * kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // K = 8 (32 bytes) per product
+          const uint32_t off = kk * 32;
+          const uint64_t a_hi = smem_desc_sw128(base + off, 16, 1024);
+          const uint64_t b_hi = smem_desc_sw128(base + kQPart + off, 16, 1024);
+          const uint64_t a_lo = smem_desc_sw128(base + kLoaded + off, 16, 1024);
+          const uint64_t b_lo = smem_desc_sw128(base + kLoaded + kQPart + off, 16, 1024);
+          mma_ss_tf32(tmem, a_hi, b_hi, idesc, (st > 0 || kk > 0) ? 1u : 0u);
+          mma_ss_tf32(tmem, a_hi, b_lo, idesc, 1u);
+          mma_ss_tf32(tmem, a_lo, b_hi, idesc, 1u);
+        }
+      }
+      mma_commit(smem_addr(&bars->empty[slot]));
+      // everything issued completes before `done` (also after a failure)
+      if (st == n_st - 1) mma_commit(smem_addr(&bars->done));
+    }
+    if (threadIdx.x == 0 && st + kMmaStages < n_st) {
+      // ------------------------------------------------------ producer
+      // the slot is free once stage st's products have read it
+      if (score_wait(smem_addr(&bars->empty[slot]), par, nullptr)) load_stage(st + kMmaStages);
+    }
+  }
+  __syncwarp();
+
+  // ------------------------------------------------------------ epilogue
+  // lane l of warp w holds query block i0 + 32 w + l: its kTileK scores go
+  // to shared memory (the ring is free: every product has read it), then
+  // each warp writes 32 rows, one row per pass, lanes along the keys
+  const bool good = __all_sync(0xffffffffu, score_wait(smem_addr(&bars->done), 0, nullptr));
+  tc_fence_after();
+  const float inv_denom = 1.0f / (sqrtf(float(d)) * __ldg(tau + (bh % H)));
+  float* stage_out = reinterpret_cast<float*>(smem);
+  __syncthreads();  // every split of the ring is over before it is reused
+  if (good) {
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+#pragma unroll
+    for (int c0 = 0; c0 < kTileK; c0 += 32) {
+      uint32_t r[32];
+      tmem_load32(tmem + lane_base + c0, r);
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        stage_out[(warp * 32 + lane) * kOutStride + c0 + c] = __uint_as_float(r[c]) * inv_denom;
+    }
+  }
+  __syncwarp();
+  if (good) {
+    const int ncols = min(kTileK, nb - j0);
+    for (int rr = 0; rr < 32; ++rr) {
+      const int row = warp * 32 + rr;
+      if (i0 + row >= nb) break;
+      float* dst = scores + (int64_t(bh) * nb + i0 + row) * nb + j0;
+#pragma unroll
+      for (int c = lane; c < kTileK; c += 32)
+        if (c < ncols) dst[c] = stage_out[row * kOutStride + c];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTileK);
   }
 }
 
@@ -305,10 +423,6 @@ __global__ void __launch_bounds__(kScoreThreads)
   const int h = (r / nb) % H;
   top_p_row<kPerLane>(scores + int64_t(r) * nb, nb, __ldg(top_p + h),
                       bits + int64_t(r) * ((nb + 31) / 32), counts + r);
-}
-
-size_t score_tile_smem_bytes(int d) {
-  return sizeof(float) * (size_t(kRowsTile) * d + 2 * size_t(kSliceFloats));
 }
 
 size_t scores_bytes(int64_t BH, int nb) {
@@ -330,7 +444,44 @@ size_t means_bytes(int64_t BH, int nb, int d) {
   return (b + 255) & ~size_t(255);
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// [rows, d] fp32 row-major, box = 32 columns (128 bytes) x box_rows rows,
+// 128-byte swizzle; rows past the end read as zeros
+bool make_means_map(CUtensorMap* map, const float* base, int64_t rows, int d, int box_rows) {
+  static EncodeTiledFn enc = nullptr;
+  if (!enc) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    enc = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(d) * 4};
+  cuuint32_t box[2] = {32, cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 }  // namespace
+
+namespace bsa {
+int take_predict_device_error() {
+  int host = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&host, g_predict_device_error, sizeof(int)) != cudaSuccess) return -1;
+  if (cudaMemcpyToSymbol(g_predict_device_error, &zero, sizeof(int)) != cudaSuccess) return -1;
+  return host;
+}
+}  // namespace bsa
 
 extern "C" size_t bsa_predict_top_p_workspace(int B, int H, int n_pad, int d, int block) {
   if (B <= 0 || H <= 0 || n_pad <= 0 || d <= 0 || block <= 0 || n_pad % block != 0) return 0;
@@ -368,21 +519,28 @@ extern "C" bsa_status bsa_predict_top_p(const void* q, const void* k, int B, int
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
+  // [q means][k means][scores][sort tables]
+  const size_t mb = means_bytes(BH, nb, d);
   float* qbar = reinterpret_cast<float*>(ws);
-  float* kbar = reinterpret_cast<float*>(ws + means_bytes(BH, nb, d));
-  float* scores = reinterpret_cast<float*>(ws + 2 * means_bytes(BH, nb, d));
-  void* scratch = ws + 2 * means_bytes(BH, nb, d) + scores_bytes(BH, nb);
+  float* kbar = reinterpret_cast<float*>(ws + mb);
+  float* scores = reinterpret_cast<float*>(ws + 2 * mb);
+  void* scratch = ws + 2 * mb + scores_bytes(BH, nb);
 
   pool_kernel<<<dim3(unsigned(nb), unsigned(BH)), kPoolThreads, 0, s>>>(
       static_cast<const uint4*>(q), static_cast<const uint4*>(k), n_valid, n_pad, d, block, qbar,
       kbar);
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
-  const size_t smem = score_tile_smem_bytes(d);
-  if (cudaFuncSetAttribute(score_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           int(smem)) != cudaSuccess)
+  CUtensorMap tq, tk;
+  const int64_t mrows = BH * nb;
+  if (!make_means_map(&tq, qbar, mrows, d, 128) || !make_means_map(&tk, kbar, mrows, d, kTileK))
     return BSA_ERR_LAUNCH;
-  score_tile_kernel<<<dim3(unsigned((nb + kRowsTile - 1) / kRowsTile), unsigned(BH)),
-                      kScoreThreads, smem, s>>>(qbar, kbar, H, nb, d, tau, scores);
+  if (cudaFuncSetAttribute(score_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(kScoreMmaSmem)) != cudaSuccess)
+    return BSA_ERR_LAUNCH;
+  score_mma_kernel<<<dim3(unsigned((nb + kTileK - 1) / kTileK), unsigned((nb + 127) / 128),
+                         unsigned(BH)),
+                     kMmaThreads, kScoreMmaSmem, s>>>(
+      tq, tk, H, nb, d, tau, scores);
   if (bsa::launch_status() != BSA_OK) return BSA_ERR_LAUNCH;
   const int rows = int(BH * nb);
   const int per_lane = (nb + 31) / 32;

@@ -234,9 +234,11 @@ bsa_status bsa_tile_unpermute(const void* in, void* out, int B, int H, int T, in
  *   s_ij = qbar_i . kbar_j / (sqrt(d) * tau[h]),  p_ij = softmax_j(s_ij)
  * Row i keeps the blocks in descending p (ties: lower j first) up to and
  * including the one where the cumulative sum reaches top_p[h]; at least one
- * block, all of them if the sum never reaches it.  Arithmetic: fp32 means,
- * fp32 FMA scores, expf; the cumulative comparison is in fp32, so a block whose
- * inclusion changes the sum by less than fp32 rounding can go either way.
+ * block, all of them if the sum never reaches it.  Arithmetic: fp32 means;
+ * scores on the tensor cores as three tf32 products per step (each mean split
+ * into a tf32 part and its remainder: fp32-level accuracy), fp32 accumulation;
+ * expf; the cumulative comparison is in fp32, so a block whose inclusion
+ * changes the sum by less than fp32 rounding can go either way.
  *
  *   q, k      [B, H, n_pad, d] bf16 in block order (as given to bsa_forward).
  *   tau, top_p  [H] fp32 device arrays.
