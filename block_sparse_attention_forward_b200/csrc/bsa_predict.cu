@@ -33,8 +33,11 @@
 //   3. topp_rows:   one warp per row: max, exp, sum, and the cut found by
 //                   bisection on the bit patterns of the (non-negative)
 //                   exponentials -- the largest T with
-//                   sum(e_j >= T) >= top_p * sum(e) -- then ties at T taken
-//                   in index order; the kept blocks are balloted into CRM words.
+//                   sum(e_j >= T) >= top_p * sum(e) -- over the whole row for
+//                   the exponent bits, then over the values that share T's
+//                   exponent only (compacted into shared memory); ties at T are
+//                   taken in index order; the kept blocks are balloted into
+//                   CRM words.
 //   4-8. the tiled count sort and the kept-block lists shared with packing.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -124,16 +127,19 @@ __device__ __forceinline__ int warp_sum_int(int x) {
 // One row, one warp.  Lane l holds blocks l + 32 k (k < kPerLane) in
 // registers; blocks past nb hold exp(-inf) = 0, which never counts.  The cut
 // is the largest bit pattern T with sum(e_j >= T) >= top_p * sum(e) (the
-// exponentials are >= 0, so patterns order like values), found by bisection
-// from the top bit over the registers (measured faster than bisecting the
-// exponent first and then only the blocks sharing it); blocks above T are kept and ties at T join in index
-// order until the cumulative sum reaches the target.  If the total never
-// reaches it (top_p >= 1, or rounding) every block is kept.  Block j = l + 32 k
-// is bit l of CRM word k.
+// exponentials lie in [0, 1], so patterns order like values and bit 30 is
+// never set), found by bisection from the top: bits 29..23 (the exponent)
+// over the whole row; then the values with T's exponent are compacted into
+// the warp's shared buffer `bucket` (kPerLane * 32 floats), those above it
+// summed once, and bits 22..0 bisect over the bucket alone.  Blocks above T
+// are kept and ties at T join in index order until the cumulative sum reaches
+// the target.  If the total never reaches it (top_p >= 1, or rounding) every
+// block is kept.  Block j = l + 32 k is bit l of CRM word k.
 template <int kPerLane>
 __device__ __forceinline__ void top_p_row(const float* __restrict__ s_row, int nb, float p_h,
                                           uint32_t* __restrict__ out,
-                                          int32_t* __restrict__ count) {
+                                          int32_t* __restrict__ count,
+                                          float* __restrict__ bucket) {
   const int lane = threadIdx.x & 31;
   const uint32_t below = (1u << lane) - 1u;
   float e[kPerLane];
@@ -154,12 +160,36 @@ __device__ __forceinline__ void top_p_row(const float* __restrict__ s_row, int n
   l = warp_sum(l);
   const float target = p_h * l;
   uint32_t T = 0;
-  for (int bit = 30; bit >= 0; --bit) {
+  for (int bit = 29; bit >= 23; --bit) {
     const uint32_t cand = T | (1u << bit);
     float sum = 0.0f;
 #pragma unroll
     for (int k = 0; k < kPerLane; ++k) sum += __float_as_uint(e[k]) >= cand ? e[k] : 0.0f;
     if (warp_sum(sum) >= target) T = cand;
+  }
+  // values above T's exponent always count; those sharing it go to the bucket
+  const uint32_t next_exp = T + (1u << 23);
+  float hi_sum = 0.0f;
+  int n_b = 0;
+#pragma unroll
+  for (int k = 0; k < kPerLane; ++k) {
+    const uint32_t eb = __float_as_uint(e[k]);
+    hi_sum += eb >= next_exp ? e[k] : 0.0f;
+    const bool in = eb >= T && eb < next_exp && lane + 32 * k < nb;
+    const uint32_t m = __ballot_sync(0xffffffffu, in);
+    if (in) bucket[n_b + __popc(m & below)] = e[k];
+    n_b += __popc(m);
+  }
+  hi_sum = warp_sum(hi_sum);
+  __syncwarp();
+  for (int bit = 22; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    float sum = 0.0f;
+    for (int i = lane; i < n_b; i += 32) {
+      const float v = bucket[i];
+      sum += __float_as_uint(v) >= cand ? v : 0.0f;
+    }
+    if (hi_sum + warp_sum(sum) >= target) T = cand;
   }
   const bool keep_all = !(l >= target);
   float above = 0.0f;
@@ -418,11 +448,13 @@ __global__ void __launch_bounds__(kScoreThreads)
     topp_rows_kernel(const float* __restrict__ scores, int H, int nb, int rows,
                      const float* __restrict__ top_p, uint32_t* __restrict__ bits,
                      int32_t* __restrict__ counts) {
+  extern __shared__ float topp_bucket[];  // [warp][kPerLane * 32]
   const int r = blockIdx.x * (kScoreThreads / 32) + (threadIdx.x >> 5);
   if (r >= rows) return;
   const int h = (r / nb) % H;
   top_p_row<kPerLane>(scores + int64_t(r) * nb, nb, __ldg(top_p + h),
-                      bits + int64_t(r) * ((nb + 31) / 32), counts + r);
+                      bits + int64_t(r) * ((nb + 31) / 32), counts + r,
+                      topp_bucket + (threadIdx.x >> 5) * kPerLane * 32);
 }
 
 size_t scores_bytes(int64_t BH, int nb) {
@@ -434,7 +466,11 @@ template <int kPerLane>
 bsa_status launch_topp_rows(int rows, cudaStream_t s, const float* scores, int H, int nb,
                             const float* top_p, uint32_t* bits, int32_t* counts) {
   const int per_cta = kScoreThreads / 32;
-  topp_rows_kernel<kPerLane><<<(rows + per_cta - 1) / per_cta, kScoreThreads, 0, s>>>(
+  const int smem = per_cta * kPerLane * 32 * int(sizeof(float));
+  if (cudaFuncSetAttribute(topp_rows_kernel<kPerLane>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return BSA_ERR_LAUNCH;
+  topp_rows_kernel<kPerLane><<<(rows + per_cta - 1) / per_cta, kScoreThreads, smem, s>>>(
       scores, H, nb, rows, top_p, bits, counts);
   return bsa::launch_status() == BSA_OK ? BSA_OK : BSA_ERR_LAUNCH;
 }
