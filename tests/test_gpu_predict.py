@@ -109,6 +109,21 @@ def test_predict_top_p_matches_oracle(cuda_ok, name, heads):
     assert 0.02 < density < 0.98
 
 
+# Tile edges of the tensor-core score kernel (128 query x 64 key blocks per
+# CTA): several batches and heads whose tiles straddle head boundaries, a key
+# count that is not a multiple of 64, d = 64 (two 32-dimension stages), and
+# two query tiles over three key tiles with a ragged last one at d = 128.
+@pytest.mark.parametrize("w", [
+    I.custom_workload("pred_b2_d64_ragged", 2, 3, 64, 5, 24, 40, 1, 8, 8, 64, 31, "bernoulli_half"),
+    I.custom_workload("pred_d128_two_row_tiles", 1, 2, 128, 9, 48, 48, 1, 8, 16, 128, 32,
+                      "bernoulli_half"),
+], ids=lambda w: w.name)
+def test_predict_top_p_tile_edges(cuda_ok, w):
+    equal, checked, density = _run(w)
+    assert equal >= 0.9 * checked, (equal, checked)
+    assert 0.02 < density < 0.98
+
+
 def test_predict_top_p_edge_parameters(cuda_ok):
     # top_p = 1 keeps everything reachable, a tiny top_p keeps one block per
     # row, a huge temperature makes rows uniform (ceil(top_p * nb) lowest blocks)
