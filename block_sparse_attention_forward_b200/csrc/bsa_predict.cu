@@ -229,14 +229,14 @@ __device__ __forceinline__ void top_p_row(const float* __restrict__ s_row, int n
 // blocks i0.., 64 key blocks j0..), two CTAs per SM (97 KB of shared memory
 // each), so that one CTA's loads and stores overlap the other's products.
 // Thread 0 issues the TMA loads of the means, 32 dimensions (one 128-byte
-// swizzle atom per row) per stage: query means 16 KB, key means 8 KB; all
-// 128 threads then split each value in place
-// into its tf32 part and write the remainder at the same offset of a parallel
-// region (the split is elementwise, so the swizzle carries over); thread 32
-// issues per stage 4 steps of K = 8, each three tcgen05.mma kind::tf32
-// products into one 128 x 64 fp32 accumulator in TMEM (hi.hi, hi.lo, lo.hi);
-// all four warps then move the accumulator (one query block per TMEM lane)
-// through shared memory to the score rows.  Rows or keys past nb (the next head's, or the
+// swizzle atom per row) per stage: query means 16 KB, key means 8 KB.  All
+// 128 threads then split each value in place into its tf32 part and write
+// the remainder at the same offset of a parallel region (the split is
+// elementwise, so the swizzle carries over).  Thread 32 issues per stage 4
+// steps of K = 8, each three tcgen05.mma kind::tf32 products into one
+// 128 x 64 fp32 accumulator in TMEM (hi.hi, hi.lo, lo.hi).  All four warps
+// then move the accumulator (one query block per TMEM lane) through shared
+// memory to the score rows.  Rows or keys past nb (the next head's, or the
 // zero fill past the last head) are computed and not stored.
 constexpr int kMmaThreads = 128;
 constexpr int kTileK = 64;                                // key blocks per CTA
@@ -345,8 +345,9 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     tma_load_2d(base, &tm_q, fbar, st * 32, bh * nb + i0);
     tma_load_2d(base + kQPart, &tm_k, fbar, st * 32, bh * nb + j0);
   };
+  int issued = 0;  // stages loaded (thread 0)
   if (threadIdx.x == 0)
-    for (int st = 0; st < n_st && st < kMmaStages; ++st) load_stage(st);
+    for (; issued < n_st && issued < kMmaStages; ++issued) load_stage(issued);
   bool ok = true;
   for (int st = 0; st < n_st; ++st) {
     const int slot = st % kMmaStages;
@@ -397,8 +398,17 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     if (threadIdx.x == 0 && st + kMmaStages < n_st) {
       // ------------------------------------------------------ producer
       // the slot is free once stage st's products have read it
-      if (score_wait(smem_addr(&bars->empty[slot]), par, nullptr)) load_stage(st + kMmaStages);
+      if (score_wait(smem_addr(&bars->empty[slot]), par, nullptr)) {
+        load_stage(st + kMmaStages);
+        ++issued;
+      }
     }
+  }
+  if (threadIdx.x == 0) {
+    // every copy issued has landed before the ring is reused or the CTA exits
+    // (already true unless a wait above ran out; bounded, ignores abort)
+    for (int st = issued > kMmaStages ? issued - kMmaStages : 0; st < issued; ++st)
+      score_wait(smem_addr(&bars->full[st % kMmaStages]), (st / kMmaStages) & 1, nullptr);
   }
   __syncwarp();
 
