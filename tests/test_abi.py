@@ -197,3 +197,29 @@ def test_pack_noalloc_rejects_oversize_on_the_host(lib, B, H, nb_q, nb_k, expect
     fake = ctypes.c_void_p(0x1000)
     assert lib.bsa_pack_mask_noalloc(fake, B, H, nb_q, nb_k, fake, fake, fake, fake, fake,
                                      None) == expect
+
+
+def test_predict_top_p_workspace_and_host_checks(lib):
+    # the workspace holds both block means, the fp32 scores and the sort's tables;
+    # every rejection below happens on the host, before any CUDA call
+    B, H, n_pad, d, block = 1, 2, 1024, 64, 64
+    nb = n_pad // block
+    need = lib.bsa_predict_top_p_workspace(B, H, n_pad, d, block)
+    assert need >= 2 * B * H * nb * d * 4 + B * H * nb * nb * 4
+    assert lib.bsa_predict_top_p_workspace(B, H, n_pad + 1, d, block) == 0  # n_pad % block
+    assert lib.bsa_predict_top_p_workspace(0, H, n_pad, d, block) == 0
+    P = ctypes.c_void_p
+    f = P(0x1000)
+
+    def call(q=f, B=B, H=H, n_valid=n_pad, n_pad=n_pad, d=d, block=block, ws=f, ws_bytes=need):
+        return lib.bsa_predict_top_p(q, f, B, H, n_valid, n_pad, d, block, f, f, f, f, f, f, f,
+                                     ws, ws_bytes, None)
+
+    assert call(q=None) == 1                                  # null input
+    assert call(n_valid=n_pad - block) == 1                   # last block would be empty
+    assert call(d=96) == 2                                    # head dim
+    assert call(n_pad=64 * 2049, n_valid=64 * 2049) == 2      # more than 2048 blocks per row
+    assert call(q=P(0x1001)) == 3                             # misaligned q
+    assert call(ws_bytes=need - 1) == 7                       # workspace too small
+    assert call(ws=None) == 7
+    assert call(ws=P(0x1008)) == 3                            # misaligned workspace
